@@ -1,0 +1,125 @@
+"""B200 (sm_100a) draft-tree round: tree_build, tree_verify_attn, tree_accept.
+
+Thin Python surface over libdtree.so (see include/dtree.h for the exact
+semantics, layouts and error behaviour of every call).  Tensors must be CUDA
+tensors; the library allocates nothing, so each call takes a workspace tensor
+(``workspace(...)`` allocates one of the right size).
+"""
+import ctypes
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import DtreeError, check, dtype_code, ptr, stream_ptr
+
+__all__ = ["Tree", "tree_build", "tree_verify_attn", "tree_accept", "markov_logits",
+           "read_status", "build_workspace_bytes", "verify_workspace_bytes",
+           "accept_workspace_bytes", "workspace", "DtreeError", "num_sms"]
+
+
+def num_sms() -> int:
+    return int(_lib.lib.dt_num_sms())
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+@dataclass
+class Tree:
+    """Device arrays of a batch of draft trees (dt_tree in the C header)."""
+    tokens: torch.Tensor      # [batch, Nmax] int32
+    parents: torch.Tensor     # [batch, Nmax] int32
+    depths: torch.Tensor      # [batch, Nmax] int32
+    ranks: torch.Tensor       # [batch, Nmax] int32
+    keys: torch.Tensor        # [batch, Nmax] float32
+    anc: torch.Tensor         # [batch, Nmax] int64 (uint64 bit patterns)
+    n_nodes: torch.Tensor     # [batch] int32
+    draft_q: Optional[torch.Tensor] = None   # [batch, Nmax+1, V] float32 (T > 0)
+
+    @staticmethod
+    def empty(batch, Nmax, V=None, stochastic=False, device="cuda"):
+        i = dict(dtype=torch.int32, device=device)
+        return Tree(
+            tokens=torch.zeros(batch, Nmax, **i), parents=torch.zeros(batch, Nmax, **i),
+            depths=torch.zeros(batch, Nmax, **i), ranks=torch.zeros(batch, Nmax, **i),
+            keys=torch.zeros(batch, Nmax, dtype=torch.float32, device=device),
+            anc=torch.zeros(batch, Nmax, dtype=torch.int64, device=device),
+            n_nodes=torch.zeros(batch, **i),
+            draft_q=(torch.zeros(batch, Nmax + 1, V, dtype=torch.float32, device=device)
+                     if stochastic else None))
+
+    def c_struct(self):
+        return _lib.DtTree(*(ctypes.c_void_p(t.data_ptr()) if t is not None else None for t in
+                             (self.tokens, self.parents, self.depths, self.ranks, self.keys,
+                              self.anc, self.n_nodes, self.draft_q)))
+
+
+def build_workspace_bytes(batch, Bk, V, r, k, Nmax) -> int:
+    return int(_lib.lib.dt_tree_build_workspace_bytes(batch, Bk, V, r, k, Nmax))
+
+
+def verify_workspace_bytes(batch, Nmax, Hq, Hkv, d, max_prefix) -> int:
+    return int(_lib.lib.dt_tree_verify_attn_workspace_bytes(batch, Nmax, Hq, Hkv, d, max_prefix))
+
+
+def accept_workspace_bytes(batch, Nmax, V) -> int:
+    return int(_lib.lib.dt_tree_accept_workspace_bytes(batch, Nmax, V))
+
+
+def tree_build(block_logits, markov_a, markov_b, root_token, n_budget, lam, *, k, Nmax, temp,
+               out: Tree, ws, calib=None, k_req=None, philox_seed=0, philox_offset=0,
+               stream=None):
+    """dt_tree_build.  block_logits [batch,Bk,V] fp32|bf16; markov_a/markov_b [V,r] bf16."""
+    batch, Bk, V = block_logits.shape
+    r = markov_a.shape[1]
+    st = out.c_struct()
+    check(_lib.lib.dt_tree_build(
+        ptr(block_logits), dtype_code(block_logits), ptr(markov_a), ptr(markov_b), r, ptr(calib),
+        ptr(root_token), ptr(n_budget), ptr(k_req), ptr(lam), batch, Bk, V, k, Nmax, float(temp),
+        philox_seed, philox_offset, ctypes.byref(st), ptr(ws), ws.numel(), stream_ptr(stream)),
+        "dt_tree_build")
+    return out
+
+
+def markov_logits(block_logits, markov_a, markov_b, req, depth, token, out, ws, stream=None):
+    """dt_markov_logits: z rows [n_rows, V] fp32 for (request, depth, token) triples."""
+    batch, Bk, V = block_logits.shape
+    check(_lib.lib.dt_markov_logits(
+        ptr(block_logits), dtype_code(block_logits), ptr(markov_a), ptr(markov_b),
+        markov_a.shape[1], batch, Bk, V, ptr(req), ptr(depth), ptr(token), req.numel(), ptr(out),
+        ptr(ws), ws.numel(), stream_ptr(stream)), "dt_markov_logits")
+    return out
+
+
+def tree_verify_attn(q, k_prefix, v_prefix, prefix_start, prefix_len, max_prefix, k_tree, v_tree,
+                     anc, n_nodes, scale, out, ws, stream=None):
+    """dt_tree_verify_attn.  q/out [batch,Nmax+1,Hq,d]; k/v_prefix [rows,Hkv,d]."""
+    batch, n1, Hq, d = q.shape
+    Hkv = k_prefix.shape[1]
+    check(_lib.lib.dt_tree_verify_attn(
+        ptr(q), ptr(k_prefix), ptr(v_prefix), ptr(prefix_start), ptr(prefix_len), int(max_prefix),
+        ptr(k_tree), ptr(v_tree), ptr(anc), ptr(n_nodes), batch, n1 - 1, Hq, Hkv, d, float(scale),
+        dtype_code(q), ptr(out), ptr(ws), ws.numel(), stream_ptr(stream)), "dt_tree_verify_attn")
+    return out
+
+
+def tree_accept(target_logits, tree: Tree, Bk, temp, acc_nodes, n_acc, bonus, ws,
+                philox_seed=0, philox_offset=0, stream=None):
+    """dt_tree_accept.  target_logits [batch,Nmax+1,V] fp32|bf16."""
+    batch, n1, V = target_logits.shape
+    st = tree.c_struct()
+    check(_lib.lib.dt_tree_accept(
+        ptr(target_logits), dtype_code(target_logits), ctypes.byref(st), batch, Bk, V, n1 - 1,
+        float(temp), philox_seed, philox_offset, ptr(acc_nodes), ptr(n_acc), ptr(bonus), ptr(ws),
+        ws.numel(), stream_ptr(stream)), "dt_tree_accept")
+    return acc_nodes, n_acc, bonus
+
+
+def read_status(ws, stream=None) -> int:
+    """Synchronise and return (then clear) the device status word of a workspace."""
+    v = ctypes.c_int32(0)
+    check(_lib.lib.dt_read_status(ptr(ws), stream_ptr(stream), ctypes.byref(v)), "dt_read_status")
+    return int(v.value)

@@ -1,0 +1,433 @@
+// Lossless acceptance walk over a verified draft tree.
+//
+// Sources: TreeSpark article, introduction (draft-then-verify with an
+// accept/reject rule that preserves the target distribution) and "lossless"
+// section (siblings sampled without replacement, residuals matched in
+// recursive rejection); PCTree summary, "setup" (greedy verification).
+//
+// Two launches.  A pre-pass over every target row of every request (row 0 =
+// root, row i+1 = node i, rows past n_nodes skipped) computes, per row chunk,
+// the argmax (T = 0) or the max and sum of exp(t / T) (T > 0).  The walk then
+// runs one CTA per request: at T = 0 it only compares child tokens with row
+// argmaxes; at T > 0 every rejected sibling costs one vocabulary-wide residual
+// pass, r <- max(p - q_j, 0), done by the whole CTA with 128-bit loads.
+#include "common.cuh"
+
+namespace dt {
+
+constexpr int kPreThreads = 256;
+constexpr int kWalkThreads = 1024;
+constexpr float kL2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float ld_logit(const void* base, int bf16, size_t i) {
+  return bf16 ? bf16_to_f32(((const uint16_t*)base)[i]) : ((const float*)base)[i];
+}
+
+struct AccParts {
+  float* pv;    // [rows_total][splits] argmax value or (T>0) max
+  int32_t* pi;  // [rows_total][splits] argmax id
+  float* ps;    // [rows_total][splits] sum exp(t/T - max)   (T > 0)
+};
+
+// Pre-pass: grid (splits, batch * (Nmax + 1)).
+template <bool STOCH>
+__global__ void __launch_bounds__(kPreThreads)
+    accept_prepass_kernel(const void* t, int tbf16, const int32_t* n_nodes, int Nmax, int V,
+                          int splits, float temp, AccParts parts) {
+  const int row_g = blockIdx.y;
+  const int b = row_g / (Nmax + 1), row = row_g % (Nmax + 1);
+  if (row > min(n_nodes[b], Nmax)) return;
+  const int chunk = ((V + splits - 1) / splits + 7) & ~7;
+  const int x0 = blockIdx.x * chunk, x1 = min(V, x0 + chunk);
+  const size_t base = (size_t)row_g * V;
+  float best = -INFINITY;
+  int32_t bid = 0x7fffffff;
+  float mx = -INFINITY, sm = 0.f;
+  const float inv_t = STOCH ? 1.f / temp : 1.f;
+  for (int x = x0 + threadIdx.x; x < x1; x += kPreThreads) {
+    const float v = ld_logit(t, tbf16, base + x);
+    if (!STOCH) {
+      if (v > best) {  // x increases within a thread: strict keeps the lower id
+        best = v;
+        bid = x;
+      }
+    } else {
+      const float s = __fdiv_rn(v, temp);
+      (void)inv_t;
+      const float d = s - mx;
+      const float ex = exp2f(-fabsf(d) * kL2e);
+      sm = d > 0.f ? fmaf(sm, ex, 1.f) : sm + ex;
+      mx = fmaxf(mx, s);
+    }
+  }
+  __shared__ float sv[kPreThreads / 32];
+  __shared__ int32_t si[kPreThreads / 32];
+  __shared__ float ss[kPreThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (!STOCH) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+      const int32_t oi = __shfl_xor_sync(0xffffffffu, bid, o);
+      if (ov > best || (ov == best && oi < bid)) {
+        best = ov;
+        bid = oi;
+      }
+    }
+    if (lane == 0) {
+      sv[warp] = best;
+      si[warp] = bid;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int w = 1; w < kPreThreads / 32; ++w)
+        if (sv[w] > best || (sv[w] == best && si[w] < bid)) {
+          best = sv[w];
+          bid = si[w];
+        }
+      parts.pv[(size_t)row_g * splits + blockIdx.x] = best;
+      parts.pi[(size_t)row_g * splits + blockIdx.x] = bid;
+    }
+  } else {
+    const float wm = warp_max(mx);
+    float ws = (mx == -INFINITY) ? 0.f : sm * exp2f((mx - wm) * kL2e);
+    ws = warp_sum(ws);
+    if (lane == 0) {
+      sv[warp] = wm;
+      ss[warp] = ws;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float m2 = -INFINITY;
+      for (int w = 0; w < kPreThreads / 32; ++w) m2 = fmaxf(m2, sv[w]);
+      float s2 = 0.f;
+      for (int w = 0; w < kPreThreads / 32; ++w)
+        if (sv[w] != -INFINITY) s2 += ss[w] * exp2f((sv[w] - m2) * kL2e);
+      parts.pv[(size_t)row_g * splits + blockIdx.x] = m2;
+      parts.ps[(size_t)row_g * splits + blockIdx.x] = s2;
+    }
+  }
+}
+
+struct WalkArgs {
+  const void* t;
+  int tbf16;
+  const int32_t* tokens;
+  const int32_t* parents;
+  const int32_t* ranks;
+  const int32_t* n_nodes;
+  const float* draft_q;
+  int Bk, V, Nmax, splits;
+  float temp;
+  uint64_t seed;
+  uint32_t offset;
+  AccParts parts;
+  float* rbuf;  // [batch][2][V] residual buffers (T > 0)
+  int32_t* acc_nodes;
+  int32_t* n_acc;
+  int32_t* bonus;
+  int32_t* status;
+};
+
+// Children of `node` in rank order (node = -1: the root's children).
+__device__ int children_of(const WalkArgs& w, int b, int n, int node, int* out) {
+  int c = 0;
+  for (int i = 0; i < n; ++i)
+    if (w.parents[(size_t)b * w.Nmax + i] == node) out[c++] = i;
+  for (int i = 1; i < c; ++i) {  // insertion sort by rank (at most k entries)
+    const int v = out[i];
+    const int rv = w.ranks[(size_t)b * w.Nmax + v];
+    int j = i - 1;
+    while (j >= 0 && w.ranks[(size_t)b * w.Nmax + out[j]] > rv) {
+      out[j + 1] = out[j];
+      --j;
+    }
+    out[j + 1] = v;
+  }
+  return c;
+}
+
+__global__ void greedy_walk_kernel(WalkArgs w) {
+  const int b = blockIdx.x;
+  if (threadIdx.x != 0) return;
+  int n = w.n_nodes[b];
+  if (n < 0 || n > w.Nmax) {
+    set_status(w.status, DT_EDEVICE);
+    n = n < 0 ? 0 : w.Nmax;
+  }
+  int kids[64];
+  int node = -1, nacc = 0;
+  int32_t a = 0;
+  while (true) {
+    const size_t rg = (size_t)b * (w.Nmax + 1) + (node + 1);
+    float best = -INFINITY;
+    a = 0x7fffffff;
+    for (int s = 0; s < w.splits; ++s) {
+      const float v = w.parts.pv[rg * w.splits + s];
+      const int32_t id = w.parts.pi[rg * w.splits + s];
+      if (v > best || (v == best && id < a)) {
+        best = v;
+        a = id;
+      }
+    }
+    const int nk = children_of(w, b, n, node, kids);
+    int next = -1;
+    for (int i = 0; i < nk; ++i)
+      if (w.tokens[(size_t)b * w.Nmax + kids[i]] == a) {
+        next = kids[i];
+        break;
+      }
+    if (next < 0 || nacc >= w.Bk) break;
+    w.acc_nodes[(size_t)b * w.Bk + nacc++] = next;
+    node = next;
+  }
+  for (int i = nacc; i < w.Bk; ++i) w.acc_nodes[(size_t)b * w.Bk + i] = -1;
+  w.n_acc[b] = nacc;
+  w.bonus[b] = a;
+}
+
+template <int NT>
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = 0.f;
+  if (warp == 0) {
+    r = lane < NT / 32 ? red[lane] : 0.f;
+    r = warp_sum(r);
+    if (lane == 0) red[0] = r;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+// Stochastic walk, one CTA per request.
+__global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ float red[32];
+  __shared__ int32_t redi[32];
+  __shared__ int kids[64];
+  __shared__ int s_nk, s_acc;
+  __shared__ float s_lse;
+  int n = w.n_nodes[b];
+  if (n < 0 || n > w.Nmax) {
+    if (tid == 0) set_status(w.status, DT_EDEVICE);
+    n = n < 0 ? 0 : w.Nmax;
+  }
+  const int V = w.V;
+  const float temp = w.temp;
+  float* rb[2] = {w.rbuf + (size_t)b * 2 * V, w.rbuf + (size_t)b * 2 * V + V};
+  int node = -1, nacc = 0;
+  int32_t bonus = 0;
+  while (true) {
+    const int row = node + 1;
+    const size_t rg = (size_t)b * (w.Nmax + 1) + row;
+    if (tid == 0) {
+      float m2 = -INFINITY;
+      for (int s = 0; s < w.splits; ++s) m2 = fmaxf(m2, w.parts.pv[rg * w.splits + s]);
+      float s2 = 0.f;
+      for (int s = 0; s < w.splits; ++s) {
+        const float mv = w.parts.pv[rg * w.splits + s];
+        if (mv != -INFINITY) s2 += w.parts.ps[rg * w.splits + s] * exp2f((mv - m2) * kL2e);
+      }
+      s_lse = m2 + logf(s2);
+      s_nk = children_of(w, b, n, node, kids);
+      s_acc = -1;
+    }
+    __syncthreads();
+    const float lse_t = s_lse;
+    const int nk = s_nk;
+    const size_t tbase = rg * V;
+    const float* q = w.draft_q + rg * V;
+    bool resid = false;  // p is softmax(t / T) until the first effective residual
+    int cur = 0;         // residual buffer holding p (unnormalised) when resid
+    float zr = 1.f;      // normaliser of the residual
+    float qn = 1.f;      // sum of q over the tokens not yet removed
+    int removed[16];
+    int n_removed = 0;
+    for (int ci = 0; ci < nk; ++ci) {
+      const int c = kids[ci];
+      const int x = w.tokens[(size_t)b * w.Nmax + c];
+      const float px = resid ? rb[cur][x] / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + x), temp) - lse_t);
+      const float qx = q[x] / qn;
+      const float u = philox_uniform(w.seed, w.offset, 1u, (uint32_t)b, (uint32_t)c, 0u, 0u);
+      if (u < px / qx) {
+        if (tid == 0) s_acc = c;
+        break;  // uniform decision: every thread computed the same values
+      }
+      // residual pass: r'(y) = max(p(y) - q_j(y), 0), q_j = q without removed tokens / qn
+      removed[n_removed++] = x;
+      float* dst = rb[cur ^ 1];
+      float zsum = 0.f, qsum = 0.f;
+      for (int y = tid; y < V; y += kWalkThreads) {
+        const float py =
+            resid ? rb[cur][y] / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + y), temp) - lse_t);
+        bool rm = false;
+        for (int i = 0; i < n_removed; ++i) rm |= (removed[i] == y);
+        const float qy = rm ? 0.f : q[y];
+        // q_j(y) uses the normaliser before this token was removed
+        const float rv = fmaxf(py - (rm && y != x ? 0.f : (y == x ? q[y] : qy)) / qn, 0.f);
+        dst[y] = rv;
+        zsum += rv;
+        if (!rm) qsum += qy;
+      }
+      zsum = block_sum<kWalkThreads>(zsum, red);
+      qsum = block_sum<kWalkThreads>(qsum, red);
+      if (zsum > 0.f) {
+        cur ^= 1;
+        zr = zsum;
+        resid = true;
+      }
+      qn = qsum;
+      __syncthreads();
+    }
+    __syncthreads();
+    const int acc = s_acc;
+    if (acc >= 0 && nacc < w.Bk) {
+      if (tid == 0) w.acc_nodes[(size_t)b * w.Bk + nacc] = acc;
+      ++nacc;
+      node = acc;
+      __syncthreads();
+      continue;
+    }
+    // bonus: exponential race argmax_y p(y) / E_y
+    float best = -INFINITY;
+    int32_t bid = 0x7fffffff;
+    for (int y = tid; y < V; y += kWalkThreads) {
+      const float py =
+          resid ? rb[cur][y] / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + y), temp) - lse_t);
+      const float u = philox_uniform(w.seed, w.offset, 2u, (uint32_t)b, (uint32_t)(node + 1), 0u,
+                                     (uint32_t)y);
+      const float sc = py / (-logf(u));
+      if (sc > best) {
+        best = sc;
+        bid = y;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+      const int32_t oi = __shfl_xor_sync(0xffffffffu, bid, o);
+      if (ov > best || (ov == best && oi < bid)) {
+        best = ov;
+        bid = oi;
+      }
+    }
+    if (lane == 0) {
+      red[warp] = best;
+      redi[warp] = bid;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      for (int i = 1; i < kWalkThreads / 32; ++i)
+        if (red[i] > best || (red[i] == best && redi[i] < bid)) {
+          best = red[i];
+          bid = redi[i];
+        }
+      bonus = bid;
+    }
+    break;
+  }
+  if (tid == 0) {
+    for (int i = nacc; i < w.Bk; ++i) w.acc_nodes[(size_t)b * w.Bk + i] = -1;
+    w.n_acc[b] = nacc;
+    w.bonus[b] = bonus;
+  }
+}
+
+}  // namespace dt
+
+using namespace dt;
+
+namespace {
+int accept_splits(int rows_total, int V) {
+  const int want = (4 * 148 + rows_total - 1) / rows_total;
+  const int most = (V + 2047) / 2048;
+  return std::max(1, std::min(want, most));
+}
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+}  // namespace
+
+extern "C" {
+
+size_t dt_tree_accept_workspace_bytes(int batch, int Nmax, int V) {
+  if (batch <= 0 || Nmax <= 0 || V <= 0) return 0;
+  const int rows = batch * (Nmax + 1);
+  const int sp = accept_splits(rows, V);
+  size_t b = kWsHeader;
+  b += align256((size_t)rows * sp * 4) * 3;
+  b += align256((size_t)batch * 2 * V * 4);
+  return b;
+}
+
+dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt, const dt_tree* tree,
+                         int batch, int Bk, int V, int Nmax, float temp, uint64_t philox_seed,
+                         uint64_t philox_offset, int32_t* d_acc_nodes, int32_t* d_n_acc,
+                         int32_t* d_bonus, void* ws, size_t ws_bytes, dt_stream stream) {
+  if (!d_target_logits || !tree || !d_acc_nodes || !d_n_acc || !d_bonus) return DT_EINVAL;
+  if (!tree->d_tokens || !tree->d_parents || !tree->d_ranks || !tree->d_n_nodes) return DT_EINVAL;
+  if (tdt != DT_F32 && tdt != DT_BF16) return DT_EINVAL;
+  if (batch < 1 || Bk < 1 || V < 1 || Nmax < 1 || !(temp >= 0.f)) return DT_EINVAL;
+  if (philox_offset >= (1ull << 32)) return DT_EINVAL;
+  if (temp > 0.f && !tree->d_draft_q) return DT_EINVAL;
+  if (batch > 1024 || Bk > 16 || Nmax > 64 || V >= (1 << 20)) return DT_EUNSUPPORTED;
+  const size_t need = dt_tree_accept_workspace_bytes(batch, Nmax, V);
+  if (!ws || ws_bytes < need) return DT_EWORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int rows = batch * (Nmax + 1);
+  const int sp = accept_splits(rows, V);
+  uint8_t* p = (uint8_t*)ws;
+  int32_t* status = (int32_t*)p;
+  p += kWsHeader;
+  AccParts parts;
+  parts.pv = (float*)p;
+  p += align256((size_t)rows * sp * 4);
+  parts.pi = (int32_t*)p;
+  p += align256((size_t)rows * sp * 4);
+  parts.ps = (float*)p;
+  p += align256((size_t)rows * sp * 4);
+  float* rbuf = (float*)p;
+  if (cudaMemsetAsync(status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
+  dim3 grid(sp, rows);
+  const int tb = tdt == DT_BF16;
+  if (temp > 0.f)
+    accept_prepass_kernel<true><<<grid, kPreThreads, 0, s>>>(d_target_logits, tb, tree->d_n_nodes,
+                                                             Nmax, V, sp, temp, parts);
+  else
+    accept_prepass_kernel<false><<<grid, kPreThreads, 0, s>>>(d_target_logits, tb,
+                                                              tree->d_n_nodes, Nmax, V, sp, temp,
+                                                              parts);
+  if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+  WalkArgs w;
+  w.t = d_target_logits;
+  w.tbf16 = tb;
+  w.tokens = tree->d_tokens;
+  w.parents = tree->d_parents;
+  w.ranks = tree->d_ranks;
+  w.n_nodes = tree->d_n_nodes;
+  w.draft_q = tree->d_draft_q;
+  w.Bk = Bk;
+  w.V = V;
+  w.Nmax = Nmax;
+  w.splits = sp;
+  w.temp = temp;
+  w.seed = philox_seed;
+  w.offset = (uint32_t)philox_offset;
+  w.parts = parts;
+  w.rbuf = rbuf;
+  w.acc_nodes = d_acc_nodes;
+  w.n_acc = d_n_acc;
+  w.bonus = d_bonus;
+  w.status = status;
+  if (temp > 0.f)
+    stoch_walk_kernel<<<batch, kWalkThreads, 0, s>>>(w);
+  else
+    greedy_walk_kernel<<<batch, 32, 0, s>>>(w);
+  if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+  return DT_OK;
+}
+
+}  // extern "C"

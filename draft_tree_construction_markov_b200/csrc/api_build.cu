@@ -1,0 +1,309 @@
+// C ABI: dt_tree_build, dt_markov_logits and the shared status helpers.
+#include <cstring>
+
+#include "build.cuh"
+
+namespace dt {
+bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows,
+                           uint32_t box_rows);
+int gemm_node_tile(int max_cols);
+cudaError_t launch_markov_gemm(int mode, bool stoch, const CUtensorMap& tmW,
+                               const CUtensorMap& tmH, const GemmArgs& a, int batch, int nt,
+                               cudaStream_t s);
+cudaError_t launch_frontier(const FrontierArgs& f, cudaStream_t s);
+cudaError_t launch_build_init(const FrontierArgs& f, const int32_t* root_token, Row* rows0,
+                              int32_t* count0, cudaStream_t s);
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Sequential carving of a workspace; every region 256-byte aligned.
+struct Carver {
+  uint8_t* base;
+  size_t off;
+  template <class T>
+  T* take(size_t count) {
+    off = align_up(off, 256);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+struct BuildLayout {
+  int32_t* status;
+  int32_t* counts;  // [0], [1] wave lists, [2] materialised rows
+  ReqState* req;
+  Cand* lists;
+  Row* rows[2];
+  Row* mat_rows;
+  uint16_t* H;
+  uint16_t* Hm;
+  float2* stats;
+  float* lv;
+  int32_t* li;
+  float* gv;
+  int32_t* gi;
+  size_t bytes;
+  int ncta_v, n_vtiles, nt, Mcap, Mcap_pad, Mmat, Mmat_pad;
+};
+
+static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k, int Nmax) {
+  BuildLayout L;
+  (void)Bk;
+  L.n_vtiles = (V + 127) / 128;
+  L.ncta_v = std::min(num_sms(), L.n_vtiles);
+  L.nt = gemm_node_tile(Nmax);
+  L.Mcap = batch * Nmax;
+  L.Mcap_pad = (int)align_up(L.Mcap, L.nt);
+  L.Mmat = batch * (Nmax + 1);
+  L.Mmat_pad = (int)align_up(L.Mmat, L.nt);
+  Carver c{(uint8_t*)ws, 0};
+  int32_t* hdr = c.take<int32_t>(kWsHeader / 4);
+  L.status = hdr;
+  L.counts = hdr + 4;
+  L.req = c.take<ReqState>(batch);
+  L.lists = c.take<Cand>((size_t)batch * Nmax);
+  L.rows[0] = c.take<Row>(L.Mcap);
+  L.rows[1] = c.take<Row>(L.Mcap);
+  L.mat_rows = c.take<Row>(L.Mmat);
+  L.H = c.take<uint16_t>((size_t)L.Mcap_pad * r);
+  L.Hm = c.take<uint16_t>((size_t)L.Mmat_pad * r);
+  const size_t np = (size_t)L.ncta_v * L.Mcap;
+  L.stats = c.take<float2>(np);
+  L.lv = c.take<float>(np * k);
+  L.li = c.take<int32_t>(np * k);
+  L.gv = c.take<float>(np * k);
+  L.gi = c.take<int32_t>(np * k);
+  L.bytes = align_up(c.off, 256);
+  return L;
+}
+
+}  // namespace dt
+
+using namespace dt;
+
+extern "C" {
+
+int dt_num_sms(void) { return num_sms(); }
+
+size_t dt_tree_build_workspace_bytes(int batch, int Bk, int V, int r, int k, int Nmax) {
+  if (batch <= 0 || Nmax <= 0 || V <= 0 || r <= 0 || k <= 0) return 0;
+  return build_layout(nullptr, batch, Bk, V, r, k, Nmax).bytes;
+}
+
+dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t* d_markov_a,
+                        const uint16_t* d_markov_b, int r, const float* d_calib,
+                        const int32_t* d_root_token, const int32_t* d_n_budget,
+                        const int32_t* d_k_req, const float* d_lambda, int batch, int Bk, int V,
+                        int k, int Nmax, float temp, uint64_t philox_seed,
+                        uint64_t philox_offset, const dt_tree* out, void* ws, size_t ws_bytes,
+                        dt_stream stream) {
+  if (!d_block_logits || !d_markov_a || !d_markov_b || !d_root_token || !d_n_budget ||
+      !d_lambda || !out)
+    return DT_EINVAL;
+  if (!out->d_tokens || !out->d_parents || !out->d_depths || !out->d_ranks || !out->d_keys ||
+      !out->d_anc || !out->d_n_nodes)
+    return DT_EINVAL;
+  if (ldt != DT_F32 && ldt != DT_BF16) return DT_EINVAL;
+  if (batch < 1 || Bk < 1 || V < 1 || k < 1 || Nmax < 1 || r < 1) return DT_EINVAL;
+  if (!(temp >= 0.f) || philox_offset >= (1ull << 32)) return DT_EINVAL;
+  if (temp > 0.f && !out->d_draft_q) return DT_EINVAL;
+  if (batch > 1024 || Bk > 16 || k > 16 || Nmax > 64 || V >= (1 << 20) || r % 16 || r > 1024)
+    return DT_EUNSUPPORTED;
+  if (k > V) return DT_EINVAL;
+  BuildLayout L = build_layout(nullptr, batch, Bk, V, r, k, Nmax);
+  if (!ws || ws_bytes < L.bytes) return DT_EWORKSPACE;
+  L = build_layout(ws, batch, Bk, V, r, k, Nmax);
+  cudaStream_t s = (cudaStream_t)stream;
+
+  CUtensorMap tmW, tmH, tmHm;
+  if (!make_tmap_bf16_kmajor(&tmW, d_markov_b, r, V, 128) ||
+      !make_tmap_bf16_kmajor(&tmH, L.H, r, L.Mcap_pad, L.nt) ||
+      !make_tmap_bf16_kmajor(&tmHm, L.Hm, r, L.Mmat_pad, L.nt))
+    return DT_ECUDA;
+
+  if (cudaMemsetAsync(L.status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
+
+  FrontierArgs f;
+  memset(&f, 0, sizeof(f));
+  f.mat_rows = L.mat_rows;
+  f.mat_count = L.counts + 2;
+  f.H = L.H;
+  f.Hm = L.Hm;
+  f.A = d_markov_a;
+  f.req = L.req;
+  f.lists = L.lists;
+  f.stats = L.stats;
+  f.lv = L.lv;
+  f.li = L.li;
+  f.gv = L.gv;
+  f.gi = L.gi;
+  f.calib = d_calib;
+  f.n_budget = d_n_budget;
+  f.k_req = d_k_req;
+  f.lambda = d_lambda;
+  f.ncta_v = L.ncta_v;
+  f.Mcap = L.Mcap;
+  f.Bk = Bk;
+  f.V = V;
+  f.r = r;
+  f.k = k;
+  f.Nmax = Nmax;
+  f.batch = batch;
+  f.temp = temp;
+  f.out = *out;
+  f.status = L.status;
+
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.L = d_block_logits;
+  g.l_bf16 = ldt == DT_BF16;
+  g.Bk = Bk;
+  g.V = V;
+  g.r = r;
+  g.k = k;
+  g.n_vtiles = L.n_vtiles;
+  g.ncta_v = L.ncta_v;
+  g.Mcap = L.Mcap;
+  g.temp = temp;
+  g.seed = philox_seed;
+  g.offset = (uint32_t)philox_offset;
+  g.stats = L.stats;
+  g.lv = L.lv;
+  g.li = L.li;
+  g.gv = L.gv;
+  g.gi = L.gi;
+  g.nmax1 = Nmax + 1;
+  g.status = L.status;
+
+  if (launch_build_init(f, d_root_token, L.rows[0], L.counts + 0, s) != cudaSuccess)
+    return DT_ECUDA;
+  const bool stoch = temp > 0.f;
+  for (int w = 0; w < Bk; ++w) {
+    const int cur = w & 1, nxt = cur ^ 1;
+    g.rows = L.rows[cur];
+    g.n_rows = L.counts + cur;
+    g.reset_count = L.counts + nxt;
+    if (launch_markov_gemm(EPI_EXPAND, stoch, tmW, tmH, g, batch, L.nt, s) != cudaSuccess)
+      return DT_ECUDA;
+    f.rows = L.rows[cur];
+    f.next_rows = L.rows[nxt];
+    f.next_count = L.counts + nxt;
+    if (launch_frontier(f, s) != cudaSuccess) return DT_ECUDA;
+  }
+  if (stoch) {
+    GemmArgs gq = g;
+    gq.rows = L.mat_rows;
+    gq.n_rows = L.counts + 2;
+    gq.reset_count = nullptr;
+    gq.Mcap = L.Mmat;
+    gq.out = out->d_draft_q;
+    if (launch_markov_gemm(EPI_QROWS, true, tmW, tmHm, gq, batch, L.nt, s) != cudaSuccess)
+      return DT_ECUDA;
+  }
+  return DT_OK;
+}
+
+// ---------------------------------------------------------------- z rows --
+namespace {
+__global__ void zrows_prep_kernel(const int32_t* req, const int32_t* depth, const int32_t* token,
+                                  int n, int V, int r, const uint16_t* A, Row* rows, uint16_t* H,
+                                  int32_t* count, int32_t* status) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    Row rw;
+    rw.b = req[i];
+    rw.depth = depth[i];
+    int t = token[i];
+    if (t < 0 || t >= V) {
+      set_status(status, DT_EDEVICE);
+      t = 0;
+      rw.b = -1;
+    }
+    rw.token = t;
+    rw.aux = i;
+    rw.path = 0;
+    rw.lse = 0.f;
+    rw.key = 0.f;
+    rows[i] = rw;
+    for (int j = 0; j < r; ++j) H[(size_t)i * r + j] = A[(size_t)t * r + j];
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *count = n;
+}
+}  // namespace
+
+size_t dt_markov_logits_workspace_bytes(int n_rows, int V, int r) {
+  (void)V;
+  if (n_rows <= 0 || r <= 0) return 0;
+  Carver c{nullptr, 0};
+  c.take<int32_t>(kWsHeader / 4);
+  c.take<Row>(n_rows);
+  c.take<uint16_t>(align_up(n_rows, 64) * r);
+  return align_up(c.off, 256);
+}
+
+dt_status dt_markov_logits(const void* d_block_logits, dt_dtype ldt, const uint16_t* d_markov_a,
+                           const uint16_t* d_markov_b, int r, int batch, int Bk, int V,
+                           const int32_t* d_req, const int32_t* d_depth, const int32_t* d_token,
+                           int n_rows, float* d_z, void* ws, size_t ws_bytes, dt_stream stream) {
+  if (!d_block_logits || !d_markov_a || !d_markov_b || !d_req || !d_depth || !d_token || !d_z)
+    return DT_EINVAL;
+  if (ldt != DT_F32 && ldt != DT_BF16) return DT_EINVAL;
+  if (n_rows < 1 || batch < 1 || Bk < 1 || V < 1 || r < 1) return DT_EINVAL;
+  if (V >= (1 << 20) || r % 16 || r > 1024 || batch > 1024 || Bk > 16) return DT_EUNSUPPORTED;
+  const size_t need = dt_markov_logits_workspace_bytes(n_rows, V, r);
+  if (!ws || ws_bytes < need) return DT_EWORKSPACE;
+  Carver c{(uint8_t*)ws, 0};
+  int32_t* hdr = c.take<int32_t>(kWsHeader / 4);
+  Row* rows = c.take<Row>(n_rows);
+  const int nt = gemm_node_tile(n_rows);
+  const int n_pad = (int)align_up(n_rows, nt);
+  uint16_t* H = c.take<uint16_t>((size_t)align_up(n_rows, 64) * r);
+  cudaStream_t s = (cudaStream_t)stream;
+  CUtensorMap tmW, tmH;
+  if (!make_tmap_bf16_kmajor(&tmW, d_markov_b, r, V, 128) ||
+      !make_tmap_bf16_kmajor(&tmH, H, r, n_pad, nt))
+    return DT_ECUDA;
+  if (cudaMemsetAsync(hdr, 0, 4, s) != cudaSuccess) return DT_ECUDA;
+  zrows_prep_kernel<<<(n_rows + 127) / 128, 128, 0, s>>>(d_req, d_depth, d_token, n_rows, V, r,
+                                                          d_markov_a, rows, H, hdr + 4, hdr);
+  if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.L = d_block_logits;
+  g.l_bf16 = ldt == DT_BF16;
+  g.Bk = Bk;
+  g.V = V;
+  g.r = r;
+  g.k = 1;
+  g.rows = rows;
+  g.n_rows = hdr + 4;
+  g.n_vtiles = (V + 127) / 128;
+  g.ncta_v = std::min(num_sms(), g.n_vtiles);
+  g.Mcap = n_rows;
+  g.out = d_z;
+  g.status = hdr;
+  if (launch_markov_gemm(EPI_ZDUMP, false, tmW, tmH, g, batch, nt, s) != cudaSuccess)
+    return DT_ECUDA;
+  return DT_OK;
+}
+
+dt_status dt_read_status(void* ws, dt_stream stream, int32_t* host_status) {
+  if (!ws || !host_status) return DT_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DT_ECUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return DT_ECUDA;
+  if (cudaMemset(ws, 0, 4) != cudaSuccess) return DT_ECUDA;
+  *host_status = v;
+  return DT_OK;
+}
+
+}  // extern "C"

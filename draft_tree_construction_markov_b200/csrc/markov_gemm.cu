@@ -1,0 +1,521 @@
+// Parent-conditioned node distributions on the 5th-generation tensor cores.
+//
+// For every GEMM column n (a tree node u with depth d and token t) and every
+// vocabulary row x:
+//   z[x][n] = L[b][d][x] + sum_rho Bm[x][rho] * A[t][rho]
+// (PCTree summary, DSpark paragraph: the Markov head biases the shared block
+// logits by the previous token; here the previous token is the node's own
+// token, i.e. the children are parent-conditioned.)
+//
+// Swap-AB tcgen05 GEMM: the vocabulary is the MMA M axis (128 rows per tile,
+// the Markov factor Bm streamed by TMA), nodes are the N axis (the gathered
+// rows A[t], also by TMA), K = r.  The fp32 accumulator lives in TMEM (double
+// buffered), and four epilogue warps per 32 node columns read it back with
+// tcgen05.ld and fuse, per node: the block-logit bias, the temperature, an
+// online max / sum-exp (log-sum-exp), the top-k of s (ties to the lower token
+// id) and, at T > 0, the Gumbel-top-k of s + G with Philox uniforms.  Each CTA
+// owns a contiguous range of vocabulary tiles and writes one partial result per
+// node; the frontier kernel merges the partials.
+#include "build.cuh"
+
+namespace dt {
+
+constexpr int kTileV = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+// U <= 1 - 2^-24 gives G = -log(-log U) <= 16.64; tokens with s + 16.75 below
+// the current k-th Gumbel key cannot enter the sample and skip the Philox draw.
+constexpr float kGumbelMax = 16.75f;
+
+template <int CPW, int NG>
+struct GemmShape {
+  static constexpr int NT = CPW * NG;  // MMA N: node columns per tile
+  static constexpr int kEpiWarps = 4 * NG;
+  static constexpr int kThreads = 32 * (2 + kEpiWarps);
+  static constexpr int kABytes = kTileV * 128;  // 128 vocab rows x 64 bf16
+  static constexpr int kBBytes = NT * 128;      // NT node rows x 64 bf16
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kTmemCols =
+      (2 * NT <= 32) ? 32 : (2 * NT <= 64) ? 64 : (2 * NT <= 128) ? 128 : (2 * NT <= 256) ? 256 : 512;
+  static_assert(NT % 16 == 0 && NT <= 256, "MMA N must be a multiple of 16, at most 256");
+};
+
+struct ColMeta {
+  int64_t bias_off;  // element offset of the node's block-logit row
+  uint32_t c1, c2;   // Philox counter words 1-2 (path id)
+  int32_t b;
+  int32_t valid;
+  float lse;
+  int32_t out_row;
+};
+
+// Host-visible SMEM size for a configuration.
+template <int CPW, int NG>
+static size_t gemm_smem_bytes(int stages, int k, bool stoch) {
+  using S = GemmShape<CPW, NG>;
+  size_t off = 1024;  // alignment slack
+  off += (size_t)stages * S::kStageBytes;
+  off += (size_t)(2 * stages + 5) * 8;          // barriers
+  off += 16;                                     // tmem slot + abort flag
+  off = (off + 15) & ~(size_t)15;
+  off += (size_t)S::NT * sizeof(ColMeta);
+  off += (size_t)S::kEpiWarps * CPW * k * 8 * (stoch ? 2 : 1);
+  off += (size_t)S::kEpiWarps * CPW * 4 * (stoch ? 2 : 1);  // list counts
+  off += (size_t)4 * S::NT * sizeof(float2);
+  return off;
+}
+
+__device__ __forceinline__ void list_insert(float* vals, int32_t* ids, int32_t* cnt, int k,
+                                            float v, int32_t id) {
+  int c = *cnt;
+  int pos = c < k ? c : k - 1;
+  while (pos > 0 && vals[pos - 1] < v) {
+    vals[pos] = vals[pos - 1];
+    ids[pos] = ids[pos - 1];
+    --pos;
+  }
+  vals[pos] = v;
+  ids[pos] = id;
+  if (c < k) *cnt = c + 1;
+}
+
+// (v1, i1) ranks before (v2, i2): larger value first, then lower id.
+__device__ __forceinline__ bool ranks_before(float v1, int32_t i1, float v2, int32_t i2) {
+  return v1 > v2 || (v1 == v2 && i1 < i2);
+}
+
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+template <int CPW, int NG, int MODE, bool STOCH>
+__global__ void __launch_bounds__(GemmShape<CPW, NG>::kThreads, 1)
+    markov_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
+                       const __grid_constant__ CUtensorMap tmH, GemmArgs a, int batch) {
+  using S = GemmShape<CPW, NG>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cx = blockIdx.x, ny = blockIdx.y;
+  const int M = min(*a.n_rows, a.Mcap);
+  if (cx == 0 && ny == 0 && threadIdx.x == 0 && a.reset_count) *a.reset_count = 0;
+  if (ny * S::NT >= M) return;  // uniform over the CTA
+
+  const int base = a.n_vtiles / a.ncta_v, extra = a.n_vtiles % a.ncta_v;
+  const int t0 = cx * base + min(cx, extra);
+  const int t1 = t0 + base + (cx < extra ? 1 : 0);
+  const int KC = (a.r + 63) >> 6;
+  const int ks_last = (((a.r - 1) & 63) >> 4) + 1;
+  const int stages = a.stages;
+  const int k = a.k;
+
+  // ---- carve shared memory
+  uint8_t* p = smem;
+  uint8_t* stage_mem = p;
+  p += (size_t)stages * S::kStageBytes;
+  uint64_t* full = (uint64_t*)p;
+  uint64_t* empty = full + stages;
+  uint64_t* tfull = empty + stages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  p = (uint8_t*)(drain + 1);
+  uint32_t* tmem_slot = (uint32_t*)p;
+  volatile int* abort_flag = (volatile int*)(p + 4);
+  p += 16;
+  p = (uint8_t*)(((uintptr_t)p + 15) & ~(uintptr_t)15);
+  ColMeta* meta = (ColMeta*)p;
+  p += S::NT * sizeof(ColMeta);
+  float* l1v = (float*)p;
+  p += (size_t)S::kEpiWarps * CPW * k * 4;
+  int32_t* l1i = (int32_t*)p;
+  p += (size_t)S::kEpiWarps * CPW * k * 4;
+  float* l2v = (float*)p;
+  int32_t* l2i = (int32_t*)p;
+  if (STOCH) {
+    p += (size_t)S::kEpiWarps * CPW * k * 4;
+    l2i = (int32_t*)p;
+    p += (size_t)S::kEpiWarps * CPW * k * 4;
+  }
+  int32_t* c1n = (int32_t*)p;
+  p += S::kEpiWarps * CPW * 4;
+  int32_t* c2n = c1n;
+  if (STOCH) {
+    c2n = (int32_t*)p;
+    p += S::kEpiWarps * CPW * 4;
+  }
+  float2* red = (float2*)p;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], S::kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmH);
+  }
+  for (int c = threadIdx.x; c < S::NT; c += blockDim.x) {
+    const int row = ny * S::NT + c;
+    ColMeta cm;
+    cm.valid = 0;
+    cm.bias_off = 0;
+    cm.c1 = cm.c2 = 0;
+    cm.b = 0;
+    cm.lse = 0.f;
+    cm.out_row = 0;
+    if (row < M) {
+      const Row r = a.rows[row];
+      if (r.b >= 0) {
+        if (r.b >= batch || r.depth < 0 || r.depth >= a.Bk) {
+          set_status(a.status, DT_EDEVICE);
+        } else {
+          cm.valid = 1;
+          cm.b = r.b;
+          cm.bias_off = ((int64_t)r.b * a.Bk + r.depth) * a.V;
+          cm.c1 = (uint32_t)r.path;
+          cm.c2 = (uint32_t)(r.path >> 32);
+          cm.lse = r.lse;
+          cm.out_row = r.aux;
+        }
+      }
+    }
+    meta[c] = cm;
+  }
+  if (MODE == EPI_EXPAND) {
+    for (int i = threadIdx.x; i < S::kEpiWarps * CPW; i += blockDim.x) {
+      c1n[i] = 0;
+      if (STOCH) c2n[i] = 0;
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::kTmemCols);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t issued = 0, last_parity = 0;  // per stage: issued at least once, parity of last issue
+      for (int t = t0; t < t1 && ok; ++t) {
+        for (int kc = 0; kc < KC; ++kc) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = stage_mem + (size_t)stage * S::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+          tma_load_2d(sa, &tmW, &full[stage], kc * 64, t * kTileV);
+          tma_load_2d(sa + S::kABytes, &tmH, &full[stage], kc * 64, ny * S::NT);
+          issued |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == stages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // let the copies already in flight land (bounded) before the CTA exits
+        const uint64_t t_start = globaltimer_ns();
+        for (int st = 0; st < stages; ++st) {
+          if (!((issued >> st) & 1)) continue;
+          while (!mbar_try_wait(&full[st], (last_parity >> st) & 1) &&
+                 globaltimer_ns() - t_start < 50000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTileV, S::NT);
+      int stage = 0;
+      uint32_t phase = 0;
+      int ab = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (int t = t0; t < t1 && ok; ++t) {
+        if (!mbar_wait(&tempty[ab], aphase ^ 1, a.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(ab * S::NT);
+        for (int kc = 0; kc < KC; ++kc) {
+          if (!mbar_wait(&full[stage], phase, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_mem + (size_t)stage * S::kStageBytes);
+          const uint64_t da = smem_desc_k_sw128(sa);
+          const uint64_t db = smem_desc_k_sw128(sa + S::kABytes);
+          const int ks = (kc == KC - 1) ? ks_last : 4;
+          for (int s = 0; s < ks; ++s)
+            tc_mma_bf16(d_tmem, da + 2 * s, db + 2 * s, idesc, (kc | s) != 0 ? 1u : 0u);
+          tc_commit(&empty[stage]);
+          if (++stage == stages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[ab]);
+        ab ^= 1;
+        if (ab == 0) aphase ^= 1;
+      }
+      // every MMA issued by this thread has completed once `drain` flips
+      tc_commit(drain);
+      const uint64_t t_start = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t_start < kWaitLimitNs) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;
+    const int q = warp & 3;  // TMEM lane quadrant accessible to this warp
+    const int g = e >> 2;    // column group
+    float m[CPW], sacc[CPW], thr[CPW], gthr[CPW];
+#pragma unroll
+    for (int j = 0; j < CPW; ++j) {
+      m[j] = -INFINITY;
+      sacc[j] = 0.f;
+      thr[j] = -INFINITY;
+      gthr[j] = -INFINITY;
+    }
+    const float temp = a.temp;
+    int ab = 0;
+    uint32_t aphase = 0;
+    for (int t = t0; t < t1; ++t) {
+      if (!mbar_wait(&tfull[ab], aphase, a.status, abort_flag)) break;
+      tc_fence_after();
+      float acc[CPW];
+      const uint32_t taddr =
+          tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * S::NT + g * CPW);
+#pragma unroll
+      for (int c = 0; c < CPW / 16; ++c) {
+        float v[16];
+        tmem_ld16(taddr + 16 * c, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[16 * c + i] = v[i];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[ab]);
+      ab ^= 1;
+      if (ab == 0) aphase ^= 1;
+
+      const int x0 = t * kTileV + 32 * q;
+      const int x = x0 + lane;
+      const bool xin = x < a.V;
+#pragma unroll
+      for (int j = 0; j < CPW; ++j) {
+        const ColMeta& cm = meta[g * CPW + j];
+        if (!cm.valid) continue;  // warp-uniform
+        float bias = 0.f;
+        if (xin)
+          bias = a.l_bf16 ? bf16_to_f32(((const uint16_t*)a.L)[cm.bias_off + x])
+                          : ((const float*)a.L)[cm.bias_off + x];
+        const float z = acc[j] + bias;
+        const float s = STOCH ? __fdiv_rn(z, temp) : z;
+        if (MODE == EPI_ZDUMP) {
+          if (xin) a.out[(size_t)cm.out_row * a.V + x] = z;
+          continue;
+        }
+        if (MODE == EPI_QROWS) {
+          if (xin) a.out[((size_t)cm.b * a.nmax1 + cm.out_row) * a.V + x] = expf(s - cm.lse);
+          continue;
+        }
+        // online max / sum of exp
+        if (xin) {
+          const float d = s - m[j];
+          const float ex = exp2f(-fabsf(d) * kLog2e);
+          sacc[j] = d > 0.f ? fmaf(sacc[j], ex, 1.f) : sacc[j] + ex;
+          m[j] = fmaxf(m[j], s);
+        }
+        const int li = (e * CPW + j);
+        // top-k of s
+        {
+          unsigned bal = __ballot_sync(0xffffffffu, xin && s > thr[j]);
+          while (bal) {
+            const int src = __ffs(bal) - 1;
+            bal &= bal - 1;
+            const float v = __shfl_sync(0xffffffffu, s, src);
+            if (v > thr[j]) {
+              if (lane == 0) list_insert(l1v + li * k, l1i + li * k, c1n + li, k, v, x0 + src);
+              __syncwarp();
+              thr[j] = (c1n[li] == k) ? l1v[li * k + k - 1] : -INFINITY;
+            }
+          }
+        }
+        if (STOCH) {
+          float gk = -INFINITY;
+          if (xin && s + kGumbelMax > gthr[j]) {
+            const float u = philox_uniform(a.seed, a.offset, 0u, (uint32_t)cm.b, cm.c1, cm.c2,
+                                           (uint32_t)x);
+            gk = s + (-logf(-logf(u)));
+          }
+          unsigned bal = __ballot_sync(0xffffffffu, gk > gthr[j]);
+          while (bal) {
+            const int src = __ffs(bal) - 1;
+            bal &= bal - 1;
+            const float v = __shfl_sync(0xffffffffu, gk, src);
+            if (v > gthr[j]) {
+              if (lane == 0) list_insert(l2v + li * k, l2i + li * k, c2n + li, k, v, x0 + src);
+              __syncwarp();
+              gthr[j] = (c2n[li] == k) ? l2v[li * k + k - 1] : -INFINITY;
+            }
+          }
+        }
+      }
+    }
+    if (MODE == EPI_EXPAND) {
+      // per-warp reduction of the softmax statistics over its 32 vocabulary rows
+#pragma unroll
+      for (int j = 0; j < CPW; ++j) {
+        const float mx = warp_max(m[j]);
+        float sv = (m[j] == -INFINITY) ? 0.f : sacc[j] * exp2f((m[j] - mx) * kLog2e);
+        sv = warp_sum(sv);
+        if (lane == 0) red[q * S::NT + g * CPW + j] = make_float2(mx, sv);
+      }
+      named_bar(1, S::kEpiWarps * 32);
+      const int et = threadIdx.x - 64;
+      for (int col = et; col < S::NT; col += S::kEpiWarps * 32) {
+        if (!meta[col].valid) continue;
+        const int row = ny * S::NT + col;
+        float mx = -INFINITY;
+        for (int qq = 0; qq < 4; ++qq) mx = fmaxf(mx, red[qq * S::NT + col].x);
+        float sv = 0.f;
+        if (mx != -INFINITY)
+          for (int qq = 0; qq < 4; ++qq) {
+            const float2 rv = red[qq * S::NT + col];
+            if (rv.x != -INFINITY) sv += rv.y * exp2f((rv.x - mx) * kLog2e);
+          }
+        const size_t pidx = (size_t)cx * a.Mcap + row;
+        a.stats[pidx] = make_float2(mx, sv);
+        // 4-way merge of the quadrant warps' sorted lists of this column
+        const int gg = col / CPW, jj = col % CPW;
+        for (int lst = 0; lst < (STOCH ? 2 : 1); ++lst) {
+          const float* LV = lst ? l2v : l1v;
+          const int32_t* LI = lst ? l2i : l1i;
+          const int32_t* LC = lst ? c2n : c1n;
+          float* OV = (lst ? a.gv : a.lv) + pidx * k;
+          int32_t* OI = (lst ? a.gi : a.li) + pidx * k;
+          int hpos[4];
+          for (int w = 0; w < 4; ++w) hpos[w] = 0;
+          for (int i = 0; i < k; ++i) {
+            int bw = -1;
+            float bv = -INFINITY;
+            int32_t bi = 0x7fffffff;
+            for (int w = 0; w < 4; ++w) {
+              const int li = (4 * gg + w) * CPW + jj;
+              if (hpos[w] < LC[li]) {
+                const float v = LV[li * k + hpos[w]];
+                const int32_t id = LI[li * k + hpos[w]];
+                if (bw < 0 || ranks_before(v, id, bv, bi)) {
+                  bw = w;
+                  bv = v;
+                  bi = id;
+                }
+              }
+            }
+            if (bw >= 0) hpos[bw]++;
+            OV[i] = bv;
+            OI[i] = bi;
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) !=
+            cudaSuccess ||
+        qres != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = (EncodeTiledFn)ptr;
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][K] (K contiguous), boxes of 64 x box_rows, 128B swizzle.
+bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows,
+                           uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {K, rows};
+  cuuint64_t strides[1] = {K * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Launch one GEMM pass.  nt_cap: 32 or 64 node columns per tile.
+template <int CPW, int NG, int MODE, bool STOCH>
+static cudaError_t launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmH, GemmArgs a,
+                              int batch, int n_node_tiles, cudaStream_t s) {
+  using SH = GemmShape<CPW, NG>;
+  auto kern = markov_gemm_kernel<CPW, NG, MODE, STOCH>;
+  // choose the deepest pipeline that fits in 220 KB
+  int stages = 8;
+  while (stages > 2 && gemm_smem_bytes<CPW, NG>(stages, a.k, STOCH) > 220 * 1024) --stages;
+  a.stages = stages;
+  const size_t smem = gemm_smem_bytes<CPW, NG>(stages, a.k, STOCH);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.ncta_v, n_node_tiles);
+  kern<<<grid, SH::kThreads, smem, s>>>(tmW, tmH, a, batch);
+  return cudaGetLastError();
+}
+
+// Node columns per tile the launcher uses for a given column capacity.
+int gemm_node_tile(int max_cols) { return max_cols <= 32 ? 32 : 64; }
+
+cudaError_t launch_markov_gemm(int mode, bool stoch, const CUtensorMap& tmW,
+                               const CUtensorMap& tmH, const GemmArgs& a, int batch, int nt,
+                               cudaStream_t s) {
+  const int ntiles = (a.Mcap + nt - 1) / nt;
+#define DT_GEMM_CASE(CPW, NG, MODE, ST)                                     \
+  if (nt == CPW * NG && mode == MODE && stoch == ST)                        \
+    return launch_cfg<CPW, NG, MODE, ST>(tmW, tmH, a, batch, ntiles, s);
+  DT_GEMM_CASE(32, 1, EPI_EXPAND, false)
+  DT_GEMM_CASE(32, 2, EPI_EXPAND, false)
+  DT_GEMM_CASE(16, 2, EPI_EXPAND, true)
+  DT_GEMM_CASE(16, 4, EPI_EXPAND, true)
+  DT_GEMM_CASE(32, 1, EPI_ZDUMP, false)
+  DT_GEMM_CASE(32, 2, EPI_ZDUMP, false)
+  DT_GEMM_CASE(32, 1, EPI_QROWS, true)
+  DT_GEMM_CASE(32, 2, EPI_QROWS, true)
+#undef DT_GEMM_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dt

@@ -1,0 +1,192 @@
+/*
+ * dtree.h -- C ABI of the B200 (sm_100a) draft-tree round library (libdtree.so).
+ *
+ * One decode round of parent-conditioned draft-tree speculative decoding:
+ *   dt_tree_build       expand a budget-N draft tree best-first from one block
+ *                       of drafter logits and a low-rank Markov head
+ *   dt_tree_verify_attn tree-masked grouped-query attention over prefix + tree
+ *   dt_tree_accept      lossless acceptance walk (greedy or recursive residual)
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named d_* are DEVICE pointers; the caller owns every buffer.
+ *     The library allocates nothing; scratch space is passed as `ws`.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL =
+ *     legacy default stream).  Arguments are validated on the host before
+ *     anything is enqueued: a call that returns DT_EINVAL / DT_EUNSUPPORTED /
+ *     DT_EWORKSPACE has enqueued nothing.
+ *   - DT_ECUDA reports a failed launch (cudaGetLastError after enqueueing).
+ *   - Device-side waits are bounded.  A wait that runs out, or an index that a
+ *     device-side check finds out of range, writes a non-zero code into the
+ *     status word inside `ws`; dt_read_status() returns it.  No kernel traps.
+ *   - Calls are stateless and re-entrant; two calls that share a `ws` must not
+ *     overlap on the device.
+ *   - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ *
+ * Random numbers: Philox4x32-10 (Salmon et al., SC'11), key = (seed lo32,
+ * seed hi32), counter word 3 = philox_offset (must be < 2^32), counter word 0
+ * = (x >> 2) | (request << 18) | (purpose << 28), output word x & 3,
+ * uniform U = ((w >> 9) + 0.5) * 2^-23 (exact in fp32).  Purposes: 0 = sibling sampling at an
+ * expanded node (words 1,2 = 64-bit path id: 4 bits per sibling rank per
+ * level, depth in bits 60..63), 1 = acceptance coin of candidate node i
+ * (word 1 = i, x = 0), 2 = bonus race at stop node s (word 1 = s + 1, root 0).
+ */
+#ifndef DTREE_H
+#define DTREE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DT_OK = 0,
+  DT_EINVAL = 1,        /* bad pointer / shape / value                       */
+  DT_EUNSUPPORTED = 2,  /* outside the supported limits listed below          */
+  DT_ECUDA = 3,         /* a CUDA call or launch failed                       */
+  DT_ETIMEOUT = 4,      /* a bounded device-side wait ran out                 */
+  DT_EWORKSPACE = 5,    /* ws is NULL or smaller than the query says          */
+  DT_EDEVICE = 6        /* a device-side range check failed                   */
+} dt_status;
+
+typedef enum { DT_F32 = 0, DT_BF16 = 1 } dt_dtype;
+
+typedef void* dt_stream; /* cudaStream_t */
+
+/* Limits: Nmax <= 64 (ancestor bitmask), 1 <= k <= 16, 1 <= Bk <= 16,
+ * batch <= 1024, V < 2^20, r a multiple of 16 in [16, 1024],
+ * head_dim in {64, 128}, Hq a multiple of Hkv. */
+
+/* Draft tree of a batch of requests; every array is caller-owned device memory.
+ * Node i of request b is element [b * Nmax + i]; nodes are in best-first pop
+ * order, which is topological (a parent precedes its children). */
+typedef struct {
+  int32_t* d_tokens;   /* [batch][Nmax] token of node i                      */
+  int32_t* d_parents;  /* [batch][Nmax] parent node index, -1 = the root     */
+  int32_t* d_depths;   /* [batch][Nmax] 1..Bk (the root has depth 0)         */
+  int32_t* d_ranks;    /* [batch][Nmax] 0-based sibling rank (sampling order)*/
+  float* d_keys;       /* [batch][Nmax] cumulative calibrated log-survival   */
+  uint64_t* d_anc;     /* [batch][Nmax] bit j set iff node j is node i or one
+                          of its ancestors                                   */
+  int32_t* d_n_nodes;  /* [batch] number of nodes of each request's tree     */
+  float* d_draft_q;    /* [batch][Nmax+1][V] fp32 draft distribution, row 0 =
+                          root, row i+1 = node i; written only when temp > 0
+                          and only for the root and nodes of depth < Bk; may
+                          be NULL when temp == 0                             */
+} dt_tree;
+
+/* ---------------------------------------------------------------- build --
+ * Expands each request's tree best-first by calibrated path survival
+ * (PCTree summary, "k=4, N=32" paragraph: shared block logits, budget N,
+ * k children per node, k = 1 gives the greedy chain; TreeSpark article,
+ * "core idea": parent-conditioned distribution from the Markov head,
+ * calibrated into an edge-acceptance estimate, path survival drives
+ * best-first expansion and per-round stopping; "lossless" section: siblings
+ * sampled without replacement).
+ *
+ * Node u of depth d < Bk with token t has children drawn from
+ *   z_u[x] = L[b][d][x] + sum_rho A[t][rho] * Bm[x][rho]      (fp32 accumulate)
+ *   s = z / T (T > 0) or z (T == 0),  lse = log sum_x exp(s_x)
+ * T == 0: children = top-k of z, ties to the lower token id.
+ * T >  0: children = Gumbel-top-k of s + G (G = -log(-log U), Philox purpose 0),
+ *         i.e. k tokens sampled without replacement, rank = sampling order.
+ * Child of rank j gets key = key(u) + min(0, alpha_{d+1} (s_(j) - lse) + beta_{d+1})
+ * with s_(j) the j-th largest s (order statistic); key(root) = 0.
+ * Nodes are taken in the order (key desc, depth asc, parent index asc, rank
+ * asc) while count < n_budget[b] and key >= fp32(log(lambda[b])).
+ *
+ *   d_block_logits [batch][Bk][V]  fp32 or bf16 (ldt)
+ *   d_markov_a     [V][r] bf16     row t = A[t]
+ *   d_markov_b     [V][r] bf16     row x = column x of B (i.e. B transposed)
+ *   d_calib        [Bk][2] fp32 (alpha, beta) for child depth 1..Bk; NULL =
+ *                  identity (1, 0); every alpha must be >= 0
+ *   d_root_token, d_n_budget (each <= Nmax, >= 0), d_k_req (each in [1, k];
+ *                  NULL = k for all), d_lambda (>= 0): [batch]
+ * Returns DT_OK after enqueueing.  Device-side range failures set DT_EDEVICE
+ * in the status word. */
+size_t dt_tree_build_workspace_bytes(int batch, int Bk, int V, int r, int k,
+                                     int Nmax);
+
+dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt,
+                        const uint16_t* d_markov_a, const uint16_t* d_markov_b,
+                        int r, const float* d_calib,
+                        const int32_t* d_root_token, const int32_t* d_n_budget,
+                        const int32_t* d_k_req, const float* d_lambda,
+                        int batch, int Bk, int V, int k, int Nmax, float temp,
+                        uint64_t philox_seed, uint64_t philox_offset,
+                        const dt_tree* out, void* ws, size_t ws_bytes,
+                        dt_stream stream);
+
+/* Diagnostic: z rows for given (request, depth, token) triples, fp32
+ * [n_rows][V] (d_z), through the same tensor-core GEMM the build uses. */
+dt_status dt_markov_logits(const void* d_block_logits, dt_dtype ldt,
+                           const uint16_t* d_markov_a,
+                           const uint16_t* d_markov_b, int r, int batch,
+                           int Bk, int V, const int32_t* d_req,
+                           const int32_t* d_depth, const int32_t* d_token,
+                           int n_rows, float* d_z, void* ws, size_t ws_bytes,
+                           dt_stream stream);
+size_t dt_markov_logits_workspace_bytes(int n_rows, int V, int r);
+
+/* ---------------------------------------------------------- verify attn --
+ * out[b][i][h] = sum_j softmax_j(scale * q[b][i][h] . k_j + mask) v_j over
+ * the columns request b's row i may see (TreeSpark article, introduction:
+ * every tree node verified in one target forward): the prefix rows
+ * [0, prefix_len[b]) of request b, the root's tree row 0, and tree row j+1 iff
+ * bit j of anc[b][i-1] is set (rows i >= 1).  Row 0 is the root; rows
+ * > n_nodes[b] are left untouched.  GQA: head h uses KV head h / (Hq/Hkv).
+ *   d_q, d_out     [batch][Nmax+1][Hq][d]
+ *   d_k_prefix, d_v_prefix  [total_prefix_rows][Hkv][d], request b's rows
+ *                  start at row d_prefix_start[b] (int64)
+ *   d_k_tree, d_v_tree      [batch][Nmax+1][Hkv][d]
+ *   d_anc [batch][Nmax] (from dt_tree), d_n_nodes [batch]
+ * dt selects fp32 or bf16 for q/k/v/out alike; accumulation is fp32. */
+size_t dt_tree_verify_attn_workspace_bytes(int batch, int Nmax, int Hq, int Hkv,
+                                           int d, int max_prefix);
+
+dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix,
+                              const void* d_v_prefix,
+                              const int64_t* d_prefix_start,
+                              const int32_t* d_prefix_len, int max_prefix,
+                              const void* d_k_tree, const void* d_v_tree,
+                              const uint64_t* d_anc, const int32_t* d_n_nodes,
+                              int batch, int Nmax, int Hq, int Hkv, int d,
+                              float scale, dt_dtype dt, void* d_out, void* ws,
+                              size_t ws_bytes, dt_stream stream);
+
+/* --------------------------------------------------------------- accept --
+ * Lossless acceptance walk from the root (TreeSpark article, introduction and
+ * "lossless" section; PCTree summary, "setup": greedy verification).
+ * T == 0: move to the child whose token is argmax of the target row (ties to
+ *   the lower id); the bonus token is that argmax where the walk stops.
+ * T >  0: at node u, p = softmax(t_u / T), q = draft row of u; children in rank
+ *   order: accept x iff U < p(x)/q(x) (Philox purpose 1); on rejection
+ *   p <- max(p - q, 0) normalised (unchanged if it sums to 0) and q <- q with x
+ *   removed, renormalised.  With no child accepted, or at a leaf, the bonus is
+ *   argmax_x p(x) / E_x, E_x = -log U'_x (Philox purpose 2).
+ *   d_target_logits [batch][Nmax+1][V] fp32 or bf16, row 0 = root, row i+1 =
+ *   node i; tree = the dt_tree of dt_tree_build (d_draft_q needed iff T > 0).
+ * Outputs (device): d_acc_nodes [batch][Bk] accepted node indices by depth
+ * (-1 padded), d_n_acc [batch], d_bonus [batch]. */
+size_t dt_tree_accept_workspace_bytes(int batch, int Nmax, int V);
+
+dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt,
+                         const dt_tree* tree, int batch, int Bk, int V,
+                         int Nmax, float temp, uint64_t philox_seed,
+                         uint64_t philox_offset, int32_t* d_acc_nodes,
+                         int32_t* d_n_acc, int32_t* d_bonus, void* ws,
+                         size_t ws_bytes, dt_stream stream);
+
+/* Synchronises `stream` and returns the status word that device code of the
+ * last call using `ws` wrote (DT_OK, DT_ETIMEOUT or DT_EDEVICE), then clears
+ * it.  `ws` is the workspace passed to that call. */
+dt_status dt_read_status(void* ws, dt_stream stream, int32_t* host_status);
+
+/* Number of streaming multiprocessors the library sizes its grids for. */
+int dt_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DTREE_H */
