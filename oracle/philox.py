@@ -12,7 +12,8 @@ Counter layout (key = (seed lo32, seed hi32), c3 = low 32 bits of offset):
   purpose 0  sibling sampling at an expanded node: c1,c2 = 64-bit path id
   purpose 1  acceptance coin of candidate node i:  c1 = i,  x = 0
   purpose 2  bonus race at stop node s:            c1 = s + 1 (root = 0)
-Uniform: U = ((w >> 8) + 0.5) * 2^-24, strictly inside (0, 1).
+Uniform: U = ((w >> 9) + 0.5) * 2^-23, strictly inside (0, 1); 23 random bits so
+that U and 1 - U are exact in fp32 as well as fp64.
 """
 import numpy as np
 
@@ -43,9 +44,9 @@ def philox4x32_10(c0, c1, c2, c3, k0, k1):
 
 
 def uniform_from_word(w):
-    """24-bit uniform strictly inside (0,1), exact in fp32 and fp64."""
+    """23-bit uniform strictly inside (0,1), exact in fp32 and fp64."""
     w = np.asarray(w, dtype=np.uint64)
-    return ((w >> np.uint64(8)).astype(np.float64) + 0.5) * 2.0 ** -24
+    return ((w >> np.uint64(9)).astype(np.float64) + 0.5) * 2.0 ** -23
 
 
 def _key(seed):
