@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Draft-tree rounds/s (build + verify + accept) on the Qwen3-4B-shaped round.
+
+One step = one decode round of one request: dt_tree_build (V=151936, B=7, k=4,
+N=32, low-rank r=256 Markov head, greedy), dt_tree_verify_attn (one layer,
+32 query / 8 KV heads, d=128, 2048-token prefix) and dt_tree_accept, on
+seeded synthetic inputs.  Rounds are replayed from CUDA graphs, one per input
+copy; four copies of every input (>300 MB, above the 126 MB L2) are rotated so
+that each round starts with a cold L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own replica (weak scaling, no collective
+in the data path); rank 0 prints one JSON line.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "qwen3_4b"
+METRIC = "draft-tree rounds/s (build+verify+accept), V=151936 B=7 N=32; % roofline"
+UNIT = "rounds/s"
+WORKLOAD_DESC = ("qwen3_4b-shaped round: V=151936, block B=7, k=4, N=32, Markov rank 256, "
+                 "bf16 block logits, greedy (T=0), verify 32q/8kv d=128 prefix 2048, batch 1")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--copies", type=int, default=4)
+    p.add_argument("--no-oracle", action="store_true", help="skip the cpu_baseline leg")
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    return rank, world, local
+
+
+# ------------------------------------------------------------------ oracle --
+def oracle_round(w, o_inputs):
+    """One round of the CPU oracle on the bench workload (build, verify, accept)."""
+    from gen import attention_inputs, target_rows
+    from oracle import accept, markov_tree, verify_attn
+    L, A64, B64 = o_inputs["L"], o_inputs["A"], o_inputs["Bt"]
+    t = markov_tree.build_tree(L, A64, B64, int(w.root[0]), w.k, w.Nmax, temp=0.0)
+    q, kp, vp, kt, vt = o_inputs["attn"]
+    verify_attn.tree_attention(q, kp, vp, kt, vt, t.anc, t.n, 1.0 / math.sqrt(w.d))
+    rows = o_inputs["target"][: t.n + 1]
+    accept.greedy_walk(t, rows)
+    return t
+
+
+def oracle_inputs(w, target):
+    from gen import attention_inputs
+    return dict(L=w.L[0].astype(np.float64), A=w.A.astype(np.float64), Bt=w.Bt.astype(np.float64),
+                attn=attention_inputs(w, w.Nmax + 1, 0), target=target.astype(np.float64))
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(w, target, budget_s=20.0, max_rounds=None):
+    oi = oracle_inputs(w, target)
+    oracle_round(w, oi)  # warm
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_round(w, oi)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or (max_rounds and n >= max_rounds):
+            break
+    return n / el, n, el
+
+
+# ---------------------------------------------------------------- clocks ----
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local):
+        vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+        self.index = vis[local].strip() if local < len(vis) else str(local)
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{local}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            c = [x.strip() for x in line.split(",")]
+            if len(c) < 9:
+                continue
+            try:
+                sm.append(float(c[1]))
+                mx = max(mx, float(c[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, c[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------- GPU ----
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def traffic_from_profile(kernel_src):
+    """DRAM bytes per launch recorded from an ncu capture, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "markov_gemm_qwen3_4b.txt")
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    vals = dict(l.split(":", 1) for l in txt.splitlines() if ":" in l and not l.startswith("#"))
+    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    if vals.get("source_sha256_16", "").strip() != sha:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_ours(args):
+    import torch
+    import draft_tree_construction_markov_b200 as dt
+    from gen import attention_inputs, make_workload, target_rows
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    bf = torch.bfloat16
+    w = make_workload(WORKLOAD, seed=rank)
+    V, Bk, N, r, k = w.V, w.Bk, w.Nmax, w.r, w.k
+    P = int(w.prefix_len[0])
+    q, kp, vp, kt, vt = attention_inputs(w, N + 1, 0)
+    host = dict(L=w.L, A=w.A, Bt=w.Bt, q=q[None], kp=kp, vp=vp, kt=kt[None], vt=vt[None])
+
+    def upload():
+        c = {nm: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(bf) for nm, a in host.items()}
+        c["root"] = torch.from_numpy(w.root).to(dev)
+        c["nb"] = torch.from_numpy(w.n_budget).to(dev)
+        c["lam"] = torch.from_numpy(w.lam).to(dev)
+        c["pstart"] = torch.zeros(1, dtype=torch.int64, device=dev)
+        c["plen"] = torch.from_numpy(w.prefix_len).to(dev)
+        return c
+
+    copies = [upload() for _ in range(args.copies)]
+    tree = dt.Tree.empty(1, N, device=dev)
+    ws_b = dt.workspace(dt.build_workspace_bytes(1, Bk, V, r, k, N), dev)
+    ws_v = dt.workspace(dt.verify_workspace_bytes(1, N, w.Hq, w.Hkv, w.d, P), dev)
+    ws_a = dt.workspace(dt.accept_workspace_bytes(1, N, V), dev)
+    attn_out = torch.empty(1, N + 1, w.Hq, w.d, dtype=bf, device=dev)
+    acc = torch.empty(1, Bk, dtype=torch.int32, device=dev)
+    nacc = torch.empty(1, dtype=torch.int32, device=dev)
+    bonus = torch.empty(1, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(w.d)
+
+    def build(c):
+        dt.tree_build(c["L"], c["A"], c["Bt"], c["root"], c["nb"], c["lam"], k=k, Nmax=N, temp=0.0,
+                      out=tree, ws=ws_b)
+
+    def verify(c):
+        dt.tree_verify_attn(c["q"], c["kp"], c["vp"], c["pstart"], c["plen"], P, c["kt"], c["vt"],
+                            tree.anc, tree.n_nodes, scale, attn_out, ws_v)
+
+    def accept_(c):
+        dt.tree_accept(c["tgt"], tree, Bk, 0.0, acc, nacc, bonus, ws_a)
+
+    # the synthetic target model scores the tree this workload builds
+    build(copies[0])
+    assert dt.read_status(ws_b) == 0
+    n = int(tree.n_nodes[0])
+    depths = tree.depths[0, :n].cpu().numpy()
+    tokens = tree.tokens[0, :n].cpu().numpy()
+    tgt = np.zeros((N + 1, V), np.float32)
+    tgt[: n + 1] = target_rows(w, 0, np.concatenate([[0], depths]),
+                               np.concatenate([w.root[:1], tokens]))
+    for c in copies:
+        c["tgt"] = torch.from_numpy(tgt[None]).to(dev).to(bf)
+
+    def round_(c):
+        build(c)
+        verify(c)
+        accept_(c)
+
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            round_(copies[i % len(copies)])
+    torch.cuda.synchronize()
+    for wsx in (ws_b, ws_v, ws_a):
+        assert dt.read_status(wsx) == 0
+    graphs = []
+    for c in copies:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            round_(c)
+        graphs.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.barrier()
+
+    # ---- timed region: K graph replays
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            graphs[i % len(graphs)].replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    ms_t = torch.tensor([ms], device=dev)
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.all_reduce(ms_t, op=tdist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    value = world * args.steps / (ms_max / 1e3)
+    for wsx in (ws_b, ws_v, ws_a):
+        assert dt.read_status(wsx) == 0
+
+    # ---- per-kernel live timing: the same rounds, eager, with the event hook
+    import ctypes
+    kprof = min(args.steps, 40)
+    cap = 64 * kprof
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap)]
+    for e in evs:
+        e.record(stream)   # materialise the handles
+    torch.cuda.synchronize()
+    ev_arr = (ctypes.c_void_p * (2 * cap))(*[e.cuda_event for e in evs])
+    kinds = (ctypes.c_int32 * cap)()
+    count = ctypes.c_int32(0)
+    dt._lib.lib.dt_set_profile_events(ev_arr, kinds, cap, ctypes.byref(count))
+    with torch.cuda.stream(stream):
+        for i in range(kprof):
+            round_(copies[i % len(copies)])
+    torch.cuda.synchronize()
+    dt._lib.lib.dt_set_profile_events(None, None, 0, None)
+    per_kind = {}
+    for i in range(count.value):
+        nm = dt._lib.KERNEL_KINDS[kinds[i]]
+        per_kind.setdefault(nm, []).append(evs[2 * i].elapsed_time(evs[2 * i + 1]))
+    launches_per_step = count.value / kprof
+    kern = {nm: {"launches_per_step": len(v) / kprof, "avg_us": 1e3 * statistics.mean(v),
+                 "us_per_step": 1e3 * sum(v) / kprof} for nm, v in per_kind.items()}
+
+    # ---- roofline of the dominant kernel (the Markov GEMM waves)
+    pk, pk_kind = peaks()
+    ncta = min(dt.num_sms(), (V + 127) // 128)
+    gemm_bytes = V * r * 2 + V * 2 + N * r * 2 + ncta * N * (8 + 8 * k)
+    g_us = kern["markov_gemm"]["avg_us"]
+    achieved = gemm_bytes / (g_us * 1e-6) / 1e9
+    roof = {"kernel": "markov_gemm (one wave: tcgen05 GEMM + fused top-k/LSE epilogue)",
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / pk["hbm_gbs"], 4), "peak_kind": pk_kind,
+            "algorithmic_bytes_per_launch": gemm_bytes,
+            "traffic": traffic_from_profile(os.path.join(
+                ROOT, "draft_tree_construction_markov_b200", "csrc", "markov_gemm.cu")),
+            "avg_launch_us": round(g_us, 3)}
+
+    # ---- end to end through the public API: pinned host inputs, copies timed
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(bf).pin_memory()
+    h_in = dict(L=pin(w.L), q=pin(q[None]), kt=pin(kt[None]), vt=pin(vt[None]), tgt=pin(tgt[None]))
+    h_root = torch.from_numpy(w.root).pin_memory()
+    h_out = {nm: torch.empty(sz, dtype=torch.int32).pin_memory()
+             for nm, sz in (("tok", (1, N)), ("par", (1, N)), ("n", (1,)), ("acc", (1, Bk)),
+                            ("nacc", (1,)), ("bonus", (1,)))}
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values()) + h_root.numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    c = copies[0]
+    ke = min(args.steps, 50)
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            for nm, t in h_in.items():
+                c[nm].copy_(t, non_blocking=True)
+            c["root"].copy_(h_root, non_blocking=True)
+            round_(c)
+            h_out["tok"].copy_(tree.tokens, non_blocking=True)
+            h_out["par"].copy_(tree.parents, non_blocking=True)
+            h_out["n"].copy_(tree.n_nodes, non_blocking=True)
+            h_out["acc"].copy_(acc, non_blocking=True)
+            h_out["nacc"].copy_(nacc, non_blocking=True)
+            h_out["bonus"].copy_(bonus, non_blocking=True)
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e3.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e = torch.tensor([e2.elapsed_time(e3)], device=dev)
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.all_reduce(ms_e, op=tdist.ReduceOp.MAX)
+    e2e = {"value": round(world * ke / (float(ms_e.item()) / 1e3), 1), "unit": UNIT,
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": ke,
+           "path": "python API (eager launches) + pinned H2D/D2H copies on the stream"}
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC, "l2": f"inputs rotated over {args.copies} copies "
+                   f"({args.copies * (2 * V * r * 2) / 1e6:.0f} MB of Markov factors > 126 MB L2)",
+                   "round": "CUDA graph per input copy", "batch_per_gpu": 1,
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "kernels": {nm: {kk: round(vv, 3) for kk, vv in d.items()} for nm, d in kern.items()},
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "e2e": e2e,
+        "clocks": clk,
+        "tree_nodes": n,
+    }
+    if rank == 0 and world == 1 and not args.no_oracle:
+        v, nr, el = time_oracle(w, tgt, budget_s=20.0)
+        out["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": blas_threads(),
+                               "kind": "oracle",
+                               "sample": f"{nr} full rounds of the same workload in {el:.1f} s "
+                                         "(numpy fp64: build + verify + accept)"}
+    if world > 1:
+        import torch.distributed as tdist
+        del graphs
+        tdist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is one CPU round of the workload."""
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    from gen import make_workload
+    from oracle import markov_tree
+    w = make_workload(WORKLOAD, seed=0)
+    t = markov_tree.build_tree(w.L[0], w.A.astype(np.float64), w.Bt.astype(np.float64),
+                               int(w.root[0]), w.k, w.Nmax)
+    from gen import target_rows
+    tgt = np.zeros((w.Nmax + 1, w.V), np.float32)
+    tgt[: t.n + 1] = target_rows(w, 0, np.concatenate([[0], t.depths]),
+                                 np.concatenate([w.root[:1], t.tokens]))
+    oi = oracle_inputs(w, tgt)
+    for _ in range(args.warmup):
+        oracle_round(w, oi)
+    # bound the whole run to a few minutes: time at most ~150 s of rounds
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(args.steps):
+        oracle_round(w, oi)
+        done += 1
+        if time.perf_counter() - t0 > 150.0:
+            break
+    el = time.perf_counter() - t0
+    v = done / el
+    sample = f"{done} of {args.steps} requested rounds (time-bounded), numpy fp64"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * el / done, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD_DESC},
+        "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}))
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)

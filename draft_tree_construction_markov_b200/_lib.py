@@ -53,6 +53,11 @@ _sig("dt_tree_accept_workspace_bytes", _sz, _i32, _i32, _i32)
 _sig("dt_tree_accept", _i32, _vp, _i32, ctypes.POINTER(DtTree), _i32, _i32, _i32, _i32, _f32,
      _u64, _u64, _vp, _vp, _vp, _vp, _sz, _vp)
 _sig("dt_read_status", _i32, _vp, _vp, ctypes.POINTER(ctypes.c_int32))
+_sig("dt_set_profile_events", None, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int32),
+     _i32, ctypes.POINTER(ctypes.c_int32))
+
+KERNEL_KINDS = ["build_init", "markov_gemm", "frontier", "draft_q", "accept_prepass",
+                "accept_walk", "attn", "attn_combine", "other"]
 
 
 class DtreeError(RuntimeError):

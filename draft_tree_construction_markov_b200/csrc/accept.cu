@@ -43,9 +43,7 @@ __global__ void __launch_bounds__(kPreThreads)
   float best = -INFINITY;
   int32_t bid = 0x7fffffff;
   float mx = -INFINITY, sm = 0.f;
-  const float inv_t = STOCH ? 1.f / temp : 1.f;
-  for (int x = x0 + threadIdx.x; x < x1; x += kPreThreads) {
-    const float v = ld_logit(t, tbf16, base + x);
+  auto consume = [&](float v, int x) {
     if (!STOCH) {
       if (v > best) {  // x increases within a thread: strict keeps the lower id
         best = v;
@@ -53,12 +51,45 @@ __global__ void __launch_bounds__(kPreThreads)
       }
     } else {
       const float s = __fdiv_rn(v, temp);
-      (void)inv_t;
       const float d = s - mx;
       const float ex = exp2f(-fabsf(d) * kL2e);
       sm = d > 0.f ? fmaf(sm, ex, 1.f) : sm + ex;
       mx = fmaxf(mx, s);
     }
+  };
+  const bool vec = tbf16 ? (V % 8 == 0) : (V % 4 == 0);
+  if (vec && tbf16) {
+    const uint4* p4 = (const uint4*)((const uint16_t*)t + base + x0);
+    const int n8 = (x1 - x0) >> 3;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < n8; i += kPreThreads) {
+      const uint4 u = p4[i];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      const int x = x0 + 8 * i;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        consume(__uint_as_float(w[h] << 16), x + 2 * h);
+        consume(__uint_as_float(w[h] & 0xFFFF0000u), x + 2 * h + 1);
+      }
+    }
+    for (int x = x0 + 8 * n8 + threadIdx.x; x < x1; x += kPreThreads)
+      consume(ld_logit(t, tbf16, base + x), x);
+  } else if (vec) {
+    const float4* p4 = (const float4*)((const float*)t + base + x0);
+    const int n4 = (x1 - x0) >> 2;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < n4; i += kPreThreads) {
+      const float4 u = p4[i];
+      const int x = x0 + 4 * i;
+      consume(u.x, x);
+      consume(u.y, x + 1);
+      consume(u.z, x + 2);
+      consume(u.w, x + 3);
+    }
+    for (int x = x0 + 4 * n4 + threadIdx.x; x < x1; x += kPreThreads)
+      consume(ld_logit(t, tbf16, base + x), x);
+  } else {
+    for (int x = x0 + threadIdx.x; x < x1; x += kPreThreads) consume(ld_logit(t, tbf16, base + x), x);
   }
   __shared__ float sv[kPreThreads / 32];
   __shared__ int32_t si[kPreThreads / 32];
@@ -129,61 +160,63 @@ struct WalkArgs {
   int32_t* status;
 };
 
-// Children of `node` in rank order (node = -1: the root's children).
-__device__ int children_of(const WalkArgs& w, int b, int n, int node, int* out) {
-  int c = 0;
-  for (int i = 0; i < n; ++i)
-    if (w.parents[(size_t)b * w.Nmax + i] == node) out[c++] = i;
-  for (int i = 1; i < c; ++i) {  // insertion sort by rank (at most k entries)
-    const int v = out[i];
-    const int rv = w.ranks[(size_t)b * w.Nmax + v];
-    int j = i - 1;
-    while (j >= 0 && w.ranks[(size_t)b * w.Nmax + out[j]] > rv) {
-      out[j + 1] = out[j];
-      --j;
-    }
-    out[j + 1] = v;
-  }
-  return c;
-}
-
+// Greedy walk: one warp per request; the tree is staged in shared memory and
+// each visited row's split partials are combined lane-parallel.
 __global__ void greedy_walk_kernel(WalkArgs w) {
-  const int b = blockIdx.x;
-  if (threadIdx.x != 0) return;
+  const int b = blockIdx.x, lane = threadIdx.x;
+  __shared__ int32_t s_tok[64], s_par[64];
   int n = w.n_nodes[b];
   if (n < 0 || n > w.Nmax) {
-    set_status(w.status, DT_EDEVICE);
+    if (lane == 0) set_status(w.status, DT_EDEVICE);
     n = n < 0 ? 0 : w.Nmax;
   }
-  int kids[64];
+  for (int i = lane; i < n; i += 32) {
+    s_tok[i] = w.tokens[(size_t)b * w.Nmax + i];
+    s_par[i] = w.parents[(size_t)b * w.Nmax + i];
+  }
+  __syncwarp();
   int node = -1, nacc = 0;
   int32_t a = 0;
   while (true) {
     const size_t rg = (size_t)b * (w.Nmax + 1) + (node + 1);
     float best = -INFINITY;
-    a = 0x7fffffff;
-    for (int s = 0; s < w.splits; ++s) {
+    int32_t bi = 0x7fffffff;
+    for (int s = lane; s < w.splits; s += 32) {
       const float v = w.parts.pv[rg * w.splits + s];
       const int32_t id = w.parts.pi[rg * w.splits + s];
-      if (v > best || (v == best && id < a)) {
+      if (v > best || (v == best && id < bi)) {
         best = v;
-        a = id;
+        bi = id;
       }
     }
-    const int nk = children_of(w, b, n, node, kids);
-    int next = -1;
-    for (int i = 0; i < nk; ++i)
-      if (w.tokens[(size_t)b * w.Nmax + kids[i]] == a) {
-        next = kids[i];
-        break;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+      const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > best || (ov == best && oi < bi)) {
+        best = ov;
+        bi = oi;
       }
+    }
+    a = bi;
+    // children of `node` carry distinct tokens: at most one matches
+    int next = -1;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + lane;
+      const bool m = i < n && s_par[i] == node && s_tok[i] == a;
+      const unsigned bal = __ballot_sync(0xffffffffu, m);
+      if (bal && next < 0) next = i0 + __ffs(bal) - 1;
+    }
     if (next < 0 || nacc >= w.Bk) break;
-    w.acc_nodes[(size_t)b * w.Bk + nacc++] = next;
+    if (lane == 0) w.acc_nodes[(size_t)b * w.Bk + nacc] = next;
+    ++nacc;
     node = next;
   }
-  for (int i = nacc; i < w.Bk; ++i) w.acc_nodes[(size_t)b * w.Bk + i] = -1;
-  w.n_acc[b] = nacc;
-  w.bonus[b] = a;
+  for (int i = nacc + lane; i < w.Bk; i += 32) w.acc_nodes[(size_t)b * w.Bk + i] = -1;
+  if (lane == 0) {
+    w.n_acc[b] = nacc;
+    w.bonus[b] = a;
+  }
 }
 
 template <int NT>
@@ -212,11 +245,18 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
   __shared__ int kids[64];
   __shared__ int s_nk, s_acc;
   __shared__ float s_lse;
+  __shared__ int32_t s_tok[64], s_par[64], s_rank[64];
   int n = w.n_nodes[b];
   if (n < 0 || n > w.Nmax) {
     if (tid == 0) set_status(w.status, DT_EDEVICE);
     n = n < 0 ? 0 : w.Nmax;
   }
+  for (int i = tid; i < n; i += kWalkThreads) {
+    s_tok[i] = w.tokens[(size_t)b * w.Nmax + i];
+    s_par[i] = w.parents[(size_t)b * w.Nmax + i];
+    s_rank[i] = w.ranks[(size_t)b * w.Nmax + i];
+  }
+  __syncthreads();
   const int V = w.V;
   const float temp = w.temp;
   float* rb[2] = {w.rbuf + (size_t)b * 2 * V, w.rbuf + (size_t)b * 2 * V + V};
@@ -225,17 +265,33 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
   while (true) {
     const int row = node + 1;
     const size_t rg = (size_t)b * (w.Nmax + 1) + row;
-    if (tid == 0) {
+    if (warp == 0) {
       float m2 = -INFINITY;
-      for (int s = 0; s < w.splits; ++s) m2 = fmaxf(m2, w.parts.pv[rg * w.splits + s]);
+      for (int s = lane; s < w.splits; s += 32) m2 = fmaxf(m2, w.parts.pv[rg * w.splits + s]);
+      m2 = warp_max(m2);
       float s2 = 0.f;
-      for (int s = 0; s < w.splits; ++s) {
+      for (int s = lane; s < w.splits; s += 32) {
         const float mv = w.parts.pv[rg * w.splits + s];
         if (mv != -INFINITY) s2 += w.parts.ps[rg * w.splits + s] * exp2f((mv - m2) * kL2e);
       }
+      s2 = warp_sum(s2);
+    if (lane == 0) {
       s_lse = m2 + logf(s2);
-      s_nk = children_of(w, b, n, node, kids);
+      int c = 0;
+      for (int i = 0; i < n; ++i)
+        if (s_par[i] == node) kids[c++] = i;
+      for (int i = 1; i < c; ++i) {  // insertion sort by rank (at most k entries)
+        const int v = kids[i];
+        int j = i - 1;
+        while (j >= 0 && s_rank[kids[j]] > s_rank[v]) {
+          kids[j + 1] = kids[j];
+          --j;
+        }
+        kids[j + 1] = v;
+      }
+      s_nk = c;
       s_acc = -1;
+    }
     }
     __syncthreads();
     const float lse_t = s_lse;
@@ -250,7 +306,7 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
     int n_removed = 0;
     for (int ci = 0; ci < nk; ++ci) {
       const int c = kids[ci];
-      const int x = w.tokens[(size_t)b * w.Nmax + c];
+      const int x = s_tok[c];
       const float px = resid ? rb[cur][x] / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + x), temp) - lse_t);
       const float qx = q[x] / qn;
       const float u = philox_uniform(w.seed, w.offset, 1u, (uint32_t)b, (uint32_t)c, 0u, 0u);
@@ -393,6 +449,8 @@ dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt, const dt_tre
   if (cudaMemsetAsync(status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
   dim3 grid(sp, rows);
   const int tb = tdt == DT_BF16;
+  {
+  ProfileScope ps(DT_K_ACCEPT_PREPASS, s);
   if (temp > 0.f)
     accept_prepass_kernel<true><<<grid, kPreThreads, 0, s>>>(d_target_logits, tb, tree->d_n_nodes,
                                                              Nmax, V, sp, temp, parts);
@@ -401,6 +459,7 @@ dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt, const dt_tre
                                                               tree->d_n_nodes, Nmax, V, sp, temp,
                                                               parts);
   if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+  }
   WalkArgs w;
   w.t = d_target_logits;
   w.tbf16 = tb;
@@ -422,6 +481,7 @@ dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt, const dt_tre
   w.n_acc = d_n_acc;
   w.bonus = d_bonus;
   w.status = status;
+  ProfileScope ps(DT_K_ACCEPT_WALK, s);
   if (temp > 0.f)
     stoch_walk_kernel<<<batch, kWalkThreads, 0, s>>>(w);
   else

@@ -1,5 +1,7 @@
 // C ABI: dt_tree_build, dt_markov_logits and the shared status helpers.
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "build.cuh"
 
@@ -13,6 +15,46 @@ cudaError_t launch_markov_gemm(int mode, bool stoch, const CUtensorMap& tmW,
 cudaError_t launch_frontier(const FrontierArgs& f, cudaStream_t s);
 cudaError_t launch_build_init(const FrontierArgs& f, const int32_t* root_token, Row* rows0,
                               int32_t* count0, cudaStream_t s);
+
+// ------------------------------------------------------------ profile hook --
+static thread_local void** g_prof_events = nullptr;
+static thread_local int32_t* g_prof_kinds = nullptr;
+static thread_local int g_prof_cap = 0;
+static thread_local int32_t* g_prof_count = nullptr;
+
+ProfileScope::ProfileScope(int kind, cudaStream_t stream) : slot(-1), s(stream) {
+  if (!g_prof_events || !g_prof_count || *g_prof_count >= g_prof_cap) return;
+  slot = (*g_prof_count)++;
+  if (g_prof_kinds) g_prof_kinds[slot] = kind;
+  cudaEventRecord((cudaEvent_t)g_prof_events[2 * slot], s);
+}
+ProfileScope::~ProfileScope() {
+  if (slot >= 0) cudaEventRecord((cudaEvent_t)g_prof_events[2 * slot + 1], s);
+}
+
+cudaError_t ensure_smem_ptr(const void* kernel, size_t bytes) {
+  struct Entry {
+    const void* k;
+    int dev;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> g(mu);
+  for (auto& e : done)
+    if (e.k == kernel && e.dev == dev && e.bytes >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  for (auto& x : done)
+    if (x.k == kernel && x.dev == dev) {
+      x.bytes = bytes;
+      return cudaSuccess;
+    }
+  done.push_back(Entry{kernel, dev, bytes});
+  return cudaSuccess;
+}
 
 int num_sms() {
   int dev = 0, n = 0;
@@ -93,6 +135,13 @@ using namespace dt;
 extern "C" {
 
 int dt_num_sms(void) { return num_sms(); }
+
+void dt_set_profile_events(void** events, int32_t* kinds, int capacity, int32_t* count) {
+  g_prof_events = events;
+  g_prof_kinds = kinds;
+  g_prof_cap = events ? capacity : 0;
+  g_prof_count = count;
+}
 
 size_t dt_tree_build_workspace_bytes(int batch, int Bk, int V, int r, int k, int Nmax) {
   if (batch <= 0 || Nmax <= 0 || V <= 0 || r <= 0 || k <= 0) return 0;
@@ -184,20 +233,29 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   g.nmax1 = Nmax + 1;
   g.status = L.status;
 
-  if (launch_build_init(f, d_root_token, L.rows[0], L.counts + 0, s) != cudaSuccess)
-    return DT_ECUDA;
+  {
+    ProfileScope ps(DT_K_BUILD_INIT, s);
+    if (launch_build_init(f, d_root_token, L.rows[0], L.counts + 0, s) != cudaSuccess)
+      return DT_ECUDA;
+  }
   const bool stoch = temp > 0.f;
   for (int w = 0; w < Bk; ++w) {
     const int cur = w & 1, nxt = cur ^ 1;
     g.rows = L.rows[cur];
     g.n_rows = L.counts + cur;
     g.reset_count = L.counts + nxt;
-    if (launch_markov_gemm(EPI_EXPAND, stoch, tmW, tmH, g, batch, L.nt, s) != cudaSuccess)
-      return DT_ECUDA;
+    {
+      ProfileScope ps(DT_K_MARKOV_GEMM, s);
+      if (launch_markov_gemm(EPI_EXPAND, stoch, tmW, tmH, g, batch, L.nt, s) != cudaSuccess)
+        return DT_ECUDA;
+    }
     f.rows = L.rows[cur];
     f.next_rows = L.rows[nxt];
     f.next_count = L.counts + nxt;
-    if (launch_frontier(f, s) != cudaSuccess) return DT_ECUDA;
+    {
+      ProfileScope ps(DT_K_FRONTIER, s);
+      if (launch_frontier(f, s) != cudaSuccess) return DT_ECUDA;
+    }
   }
   if (stoch) {
     GemmArgs gq = g;
@@ -206,6 +264,7 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
     gq.reset_count = nullptr;
     gq.Mcap = L.Mmat;
     gq.out = out->d_draft_q;
+    ProfileScope ps(DT_K_DRAFT_Q, s);
     if (launch_markov_gemm(EPI_QROWS, true, tmW, tmHm, gq, batch, L.nt, s) != cudaSuccess)
       return DT_ECUDA;
   }

@@ -208,4 +208,20 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }
 
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t ensure_smem_ptr(const void* kernel, size_t bytes);
+template <class K>
+inline cudaError_t ensure_smem(K* kernel, size_t bytes) {
+  return ensure_smem_ptr(reinterpret_cast<const void*>(kernel), bytes);
+}
+
+// ---------------------------------------------------------- profiling hook --
+// Host side: brackets a launch with caller-owned events when the hook is set.
+struct ProfileScope {
+  int slot;
+  cudaStream_t s;
+  ProfileScope(int kind, cudaStream_t stream);
+  ~ProfileScope();
+};
+
 }  // namespace dt

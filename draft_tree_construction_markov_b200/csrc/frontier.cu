@@ -16,7 +16,7 @@
 
 namespace dt {
 
-constexpr int kFrontierThreads = 256;
+constexpr int kFrontierThreads = 1024;
 constexpr float kLog2eF = 1.4426950408889634f;
 
 __device__ __forceinline__ uint64_t sort_key(const Cand& c, int idx) {
@@ -47,9 +47,10 @@ __device__ __forceinline__ void warp_best(float& v, int32_t& id) {
   }
 }
 
-// k rounds: each picks the best entry ranked strictly after the previous pick.
-__device__ void merge_topk(const float* lv, const int32_t* li, int ncta, size_t Mcap, int row,
-                           int k, int kb, float* out_v, int32_t* out_i) {
+// Exact fallback: kb rounds, each picks the best entry ranked strictly after
+// the previous pick (used only when ties overflow the candidate buffer).
+__device__ void merge_topk_slow(const float* lv, const int32_t* li, int ncta, size_t Mcap, int row,
+                                int k, int kb, float* out_v, int32_t* out_i) {
   const int lane = threadIdx.x & 31;
   float pv = INFINITY;
   int32_t pi = -1;
@@ -80,6 +81,78 @@ __device__ void merge_topk(const float* lv, const int32_t* li, int ncta, size_t 
   }
 }
 
+constexpr int kMergeCap = 128;  // candidates per warp that survive the threshold
+
+// Top-kb over the per-CTA sorted top-k lists of one row, by one warp.
+// Threshold: the largest kb-th value of any single list; every member of the
+// global top-kb is >= it (that list alone holds kb values >= it), and usually
+// only a handful of entries pass.  buf: kMergeCap (value, id) pairs of smem.
+__device__ void merge_topk(const float* lv, const int32_t* li, int ncta, size_t Mcap, int row,
+                           int k, int kb, float* out_v, int32_t* out_i, float* bv_s,
+                           int32_t* bi_s, int* bcount) {
+  const int lane = threadIdx.x & 31;
+  float tau = -INFINITY;
+  for (int c = lane; c < ncta; c += 32) tau = fmaxf(tau, lv[((size_t)c * Mcap + row) * k + kb - 1]);
+  tau = warp_max(tau);
+  if (lane == 0) *bcount = 0;
+  __syncwarp();
+  for (int c = lane; c < ncta; c += 32) {
+    const size_t base = ((size_t)c * Mcap + row) * k;
+    for (int i = 0; i < k; ++i) {
+      const float v = lv[base + i];
+      if (!(v >= tau)) break;  // sorted descending
+      const int slot = atomicAdd(bcount, 1);
+      if (slot < kMergeCap) {
+        bv_s[slot] = v;
+        bi_s[slot] = li[base + i];
+      }
+    }
+  }
+  __syncwarp();
+  const int nb = *bcount;
+  if (nb > kMergeCap) {
+    merge_topk_slow(lv, li, ncta, Mcap, row, k, kb, out_v, out_i);
+    return;
+  }
+  // kb rounds of a warp argmax over the buffer (at most 4 entries per lane)
+  float ev[kMergeCap / 32];
+  int32_t ei[kMergeCap / 32];
+#pragma unroll
+  for (int t = 0; t < kMergeCap / 32; ++t) {
+    const int sidx = lane + 32 * t;
+    ev[t] = sidx < nb ? bv_s[sidx] : -INFINITY;
+    ei[t] = sidx < nb ? bi_s[sidx] : 0x7fffffff;
+  }
+  for (int j = 0; j < kb; ++j) {
+    int bt = 0;
+#pragma unroll
+    for (int t = 1; t < kMergeCap / 32; ++t)
+      if (ev[t] > ev[bt] || (ev[t] == ev[bt] && ei[t] < ei[bt])) bt = t;
+    float wv = ev[0];
+    int32_t wi = ei[0];
+#pragma unroll
+    for (int t = 1; t < kMergeCap / 32; ++t)
+      if (t == bt) {
+        wv = ev[t];
+        wi = ei[t];
+      }
+    const float mv = wv;
+    const int32_t mi = wi;
+    warp_best(wv, wi);
+#pragma unroll
+    for (int t = 0; t < kMergeCap / 32; ++t)
+      if (t == bt && mv == wv && mi == wi) {
+        ev[t] = -INFINITY;
+        ei[t] = 0x7fffffff;
+      }
+    if (lane == 0) {
+      out_v[j] = wv;
+      out_i[j] = wi;
+    }
+  }
+  __syncwarp();
+}
+
 __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs f) {
   extern __shared__ __align__(16) uint8_t fsm[];
   const int b = blockIdx.x;
@@ -91,6 +164,9 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
   __shared__ int s_kb, s_nb;
   __shared__ uint64_t s_anc[64];
   __shared__ int32_t s_par[64];
+  __shared__ float s_mv[kFrontierThreads / 32][kMergeCap];
+  __shared__ int32_t s_mi[kFrontierThreads / 32][kMergeCap];
+  __shared__ int s_mc[kFrontierThreads / 32];
   if (tid == 0) {
     st = f.req[b];
     int kb = f.k_req ? f.k_req[b] : f.k;
@@ -114,12 +190,10 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
   const int rows_n = st.row_count;
   const int n_old = st.n_list;
   const int cap = Nmax + Nmax * k;  // list + children of at most Nmax expanded nodes
-  int sortn = 1;
-  while (sortn < cap) sortn <<= 1;
   Cand* cands = (Cand*)fsm;                                   // [cap]
   Cand* sorted = cands + cap;                                 // [Nmax]
-  uint64_t* keys = (uint64_t*)(sorted + Nmax);                // [sortn]
-  float* r_lse = (float*)(keys + sortn);                      // [Nmax]
+  uint64_t* keys = (uint64_t*)(sorted + Nmax);                // [cap]
+  float* r_lse = (float*)(keys + cap);                        // [Nmax]
   float* r_lq = r_lse + Nmax;                                 // [Nmax][k]
   int32_t* r_tok = (int32_t*)(r_lq + Nmax * k);               // [Nmax][k]
   float* r_sv = (float*)(r_tok + Nmax * k);                   // scratch [Nmax][k]
@@ -141,9 +215,11 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
     sv = warp_sum(sv);
     const float lse = mx + logf(sv);
     // order statistics of s (and, at T = 0, the children themselves)
-    merge_topk(f.lv, f.li, f.ncta_v, f.Mcap, row, k, kb, r_sv + e * k, r_si + e * k);
+    merge_topk(f.lv, f.li, f.ncta_v, f.Mcap, row, k, kb, r_sv + e * k, r_si + e * k, s_mv[warp],
+               s_mi[warp], &s_mc[warp]);
     if (f.temp > 0.f)
-      merge_topk(f.gv, f.gi, f.ncta_v, f.Mcap, row, k, kb, r_lq + e * k, r_tok + e * k);
+      merge_topk(f.gv, f.gi, f.ncta_v, f.Mcap, row, k, kb, r_lq + e * k, r_tok + e * k,
+                 s_mv[warp], s_mi[warp], &s_mc[warp]);
     __syncwarp();
     if (lane == 0) {
       r_lse[e] = lse;
@@ -204,36 +280,26 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
         if (cands[p].serial == rw.aux) cands[p].lse = r_lse[tid];
     }
   }
-  // 3. sort list + candidates by the total order; drop keys below log(lambda)
+  // 3. rank list + candidates by the total order (keys are unique: the low
+  // bits hold the slot); keys below log(lambda) are dropped
   const int n_all = n_old + n_new;
   const float thr = s_thr;
-  for (int i = tid; i < sortn; i += kFrontierThreads)
-    keys[i] = (i < n_all && cands[i].key >= thr) ? sort_key(cands[i], i) : ~0ull;
+  for (int i = tid; i < n_all; i += kFrontierThreads)
+    keys[i] = (cands[i].key >= thr) ? sort_key(cands[i], i) : ~0ull;
+  if (tid == 0) s_n_keep = 0;
   __syncthreads();
-  for (int size = 2; size <= sortn; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < sortn / 2; i += kFrontierThreads) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool up = ((lo & size) == 0);
-        const uint64_t a = keys[lo], c = keys[hi];
-        if ((a > c) == up) {
-          keys[lo] = c;
-          keys[hi] = a;
-        }
-      }
-      __syncthreads();
+  for (int i = tid; i < n_all; i += kFrontierThreads) {
+    const uint64_t ki = keys[i];
+    if (ki == ~0ull) continue;
+    int rank = 0;
+    for (int j = 0; j < n_all; ++j) rank += keys[j] < ki;
+    if (rank < s_nb) {
+      sorted[rank] = cands[i];
+      atomicAdd(&s_n_keep, 1);
     }
-  }
-  if (tid == 0) {
-    int nk = 0;
-    while (nk < s_nb && nk < sortn && keys[nk] != ~0ull) ++nk;
-    s_n_keep = nk;
   }
   __syncthreads();
   const int n_keep = s_n_keep;
-  for (int i = tid; i < n_keep; i += kFrontierThreads) sorted[i] = cands[keys[i] & 0xFFFF];
-  __syncthreads();
 
   // 4. schedule the next wave: kept nodes not yet expanded, depth < Bk
   if (tid == 0) {
@@ -362,7 +428,9 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
 // Wave 1: every request with a non-empty budget expands its root.
 __global__ void build_init_kernel(FrontierArgs f, const int32_t* root_token, Row* rows0,
                                   int32_t* count0) {
-  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < f.batch; b += gridDim.x * blockDim.x) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int b = blockIdx.x * wpb + (threadIdx.x >> 5); b < f.batch; b += gridDim.x * wpb) {
     ReqState st;
     st.n_list = 0;
     st.serial_next = 0;
@@ -372,7 +440,7 @@ __global__ void build_init_kernel(FrontierArgs f, const int32_t* root_token, Row
     st.root_lse = 0.f;
     int root = root_token[b];
     if (root < 0 || root >= f.V) {
-      set_status(f.status, DT_EDEVICE);
+      if (lane == 0) set_status(f.status, DT_EDEVICE);
       root = 0;
     }
     st.pad[0] = root;
@@ -390,12 +458,14 @@ __global__ void build_init_kernel(FrontierArgs f, const int32_t* root_token, Row
       rw.b = -1;
       st.done = 1;
       st.row_count = 0;
-      f.out.d_n_nodes[b] = 0;
+      if (lane == 0) f.out.d_n_nodes[b] = 0;
     } else {
-      gather_row(f.H + (size_t)b * f.r, f.A, root, f.r, 0, 1);
+      gather_row(f.H + (size_t)b * f.r, f.A, root, f.r, lane, 32);
     }
-    rows0[b] = rw;
-    f.req[b] = st;
+    if (lane == 0) {
+      rows0[b] = rw;
+      f.req[b] = st;
+    }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     *count0 = f.batch;
@@ -405,16 +475,13 @@ __global__ void build_init_kernel(FrontierArgs f, const int32_t* root_token, Row
 
 size_t frontier_smem_bytes(int Nmax, int k) {
   const int cap = Nmax + Nmax * k;
-  int sortn = 1;
-  while (sortn < cap) sortn <<= 1;
-  return (size_t)cap * sizeof(Cand) + (size_t)Nmax * sizeof(Cand) + (size_t)sortn * 8 +
+  return (size_t)cap * sizeof(Cand) + (size_t)Nmax * sizeof(Cand) + (size_t)cap * 8 +
          (size_t)Nmax * 4 + (size_t)Nmax * k * 4 * 4;
 }
 
 cudaError_t launch_frontier(const FrontierArgs& f, cudaStream_t s) {
   const size_t smem = frontier_smem_bytes(f.Nmax, f.k);
-  cudaError_t e = cudaFuncSetAttribute(frontier_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_smem(frontier_kernel, smem);
   if (e != cudaSuccess) return e;
   frontier_kernel<<<f.batch, kFrontierThreads, smem, s>>>(f);
   return cudaGetLastError();
@@ -422,7 +489,7 @@ cudaError_t launch_frontier(const FrontierArgs& f, cudaStream_t s) {
 
 cudaError_t launch_build_init(const FrontierArgs& f, const int32_t* root_token, Row* rows0,
                               int32_t* count0, cudaStream_t s) {
-  build_init_kernel<<<(f.batch + 255) / 256, 256, 0, s>>>(f, root_token, rows0, count0);
+  build_init_kernel<<<(f.batch + 7) / 8, 256, 0, s>>>(f, root_token, rows0, count0);
   return cudaGetLastError();
 }
 

@@ -257,8 +257,13 @@ __global__ void __launch_bounds__(512) attn_bf16_kernel(AttnArgs a) {
   }
 }
 
-// Merge the column splits: grid (batch * (Nmax+1), Hq), D threads.
+constexpr int kMaxSplits = 512;
+
+// Merge the column splits: grid (batch * (Nmax+1), Hq), 128 threads.
 __global__ void attn_combine_kernel(AttnArgs a) {
+  __shared__ float s_w[kMaxSplits];
+  __shared__ float s_l[kMaxSplits];
+  __shared__ float s_red[2];
   const int b = blockIdx.x / (a.Nmax + 1), i = blockIdx.x % (a.Nmax + 1);
   const int h = blockIdx.y;
   if (i > min(a.n_nodes[b], a.Nmax)) return;
@@ -267,25 +272,34 @@ __global__ void attn_combine_kernel(AttnArgs a) {
   const int rb = rho / a.rows_per_cta, rl = rho % a.rows_per_cta;
   const int P = min(max(a.plen[b], 0), a.max_prefix);
   const int C = P + min(max(a.n_nodes[b], 0), a.Nmax) + 1;
-  const int used = (C + a.cols_per_split - 1) / a.cols_per_split;
-  float mx = -INFINITY;
-  for (int s = 0; s < used; ++s) {
-    const size_t pb = (((size_t)s * a.batch + b) * a.Hkv + kvh) * (size_t)(a.n_rblocks * a.rpad) +
-                      rb * a.rows_per_cta + rl;
-    mx = fmaxf(mx, a.part_ml[pb].x);
+  const int used = min((C + a.cols_per_split - 1) / a.cols_per_split, kMaxSplits);
+  const size_t split_stride = (size_t)a.batch * a.Hkv * a.n_rblocks * a.rpad;
+  const size_t pb0 = ((size_t)b * a.Hkv + kvh) * (size_t)(a.n_rblocks * a.rpad) +
+                     rb * a.rows_per_cta + rl;
+  for (int s = threadIdx.x; s < used; s += blockDim.x) {
+    const float2 ml = a.part_ml[pb0 + s * split_stride];
+    s_w[s] = ml.x;
+    s_l[s] = ml.y;
   }
-  for (int dd = threadIdx.x; dd < a.d; dd += blockDim.x) {
-    float acc = 0.f, l = 0.f;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float mx = -INFINITY;
+    for (int s = 0; s < used; ++s) mx = fmaxf(mx, s_w[s]);
+    float l = 0.f;
     for (int s = 0; s < used; ++s) {
-      const size_t pb = (((size_t)s * a.batch + b) * a.Hkv + kvh) * (size_t)(a.n_rblocks * a.rpad) +
-                        rb * a.rows_per_cta + rl;
-      const float2 ml = a.part_ml[pb];
-      if (ml.x == -INFINITY) continue;
-      const float w = exp2f(ml.x - mx);
-      acc += w * a.part_o[pb * a.d + dd];
-      l += w * ml.y;
+      const float wgt = s_w[s] == -INFINITY ? 0.f : exp2f(s_w[s] - mx);
+      s_w[s] = wgt;
+      l += wgt * s_l[s];
     }
-    const float v = acc / l;
+    s_red[0] = l;
+  }
+  __syncthreads();
+  const float inv_l = 1.f / s_red[0];
+  for (int dd = threadIdx.x; dd < a.d; dd += blockDim.x) {
+    float acc = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < used; ++s) acc += s_w[s] * a.part_o[(pb0 + s * split_stride) * a.d + dd];
+    const float v = acc * inv_l;
     const size_t oi = (((size_t)b * (a.Nmax + 1) + i) * a.Hq + h) * a.d + dd;
     if (a.out_bf16)
       ((uint16_t*)a.out)[oi] = (uint16_t)(pack_bf16(v, 0.f) & 0xFFFF);
@@ -388,7 +402,7 @@ static AttnPlan attn_plan(int batch, int Nmax, int Hq, int Hkv, int d, int max_p
   want = std::max(1, std::min(want, chunks));
   const int chunks_per = (chunks + want - 1) / want;
   p.cols_per_split = chunks_per * kChunk;
-  p.splits = (chunks + chunks_per - 1) / chunks_per;
+  p.splits = (chunks + chunks_per - 1) / chunks_per;  // at most 2 * 148 <= kMaxSplits
   const size_t rows = (size_t)p.splits * batch * Hkv * p.n_rblocks * p.rpad;
   p.part_o_bytes = rows * d * 4;
   p.part_ml_bytes = rows * 8;
@@ -461,27 +475,29 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const voi
     const int max_cols = max_prefix + Nmax + 1;
     const size_t smem = (size_t)max_cols * 4;
     if (smem > 200 * 1024) return DT_EUNSUPPORTED;
-    if (cudaFuncSetAttribute(attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (ensure_smem(attn_f32_kernel, smem) != cudaSuccess)
       return DT_ECUDA;
+    ProfileScope ps(DT_K_ATTN, s);
     attn_f32_kernel<<<dim3(batch * (Nmax + 1), Hq), 128, smem, s>>>(a, max_cols);
     return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ECUDA;
   }
   const size_t smem = ((size_t)p.rows_per_cta + 2 * kChunk) * (d + 8) * 2;
   dim3 grid(p.splits, Hkv, batch * p.n_rblocks);
   const int threads = 32 * std::max(p.warps, 4);
+  {
+  ProfileScope ps(DT_K_ATTN, s);
   if (d == 128) {
-    if (cudaFuncSetAttribute(attn_bf16_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (ensure_smem(attn_bf16_kernel<128>, smem) != cudaSuccess)
       return DT_ECUDA;
     attn_bf16_kernel<128><<<grid, threads, smem, s>>>(a);
   } else {
-    if (cudaFuncSetAttribute(attn_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (ensure_smem(attn_bf16_kernel<64>, smem) != cudaSuccess)
       return DT_ECUDA;
     attn_bf16_kernel<64><<<grid, threads, smem, s>>>(a);
   }
   if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+  }
+  ProfileScope ps(DT_K_ATTN_COMBINE, s);
   attn_combine_kernel<<<dim3(batch * (Nmax + 1), Hq), 128, 0, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ECUDA;
 }

@@ -72,8 +72,8 @@ typedef struct {
   int32_t* d_n_nodes;  /* [batch] number of nodes of each request's tree     */
   float* d_draft_q;    /* [batch][Nmax+1][V] fp32 draft distribution, row 0 =
                           root, row i+1 = node i; written only when temp > 0
-                          and only for the root and nodes of depth < Bk; may
-                          be NULL when temp == 0                             */
+                          and only for the root and nodes of depth < Bk of
+                          non-empty trees; may be NULL when temp == 0        */
 } dt_tree;
 
 /* ---------------------------------------------------------------- build --
@@ -185,6 +185,28 @@ dt_status dt_read_status(void* ws, dt_stream stream, int32_t* host_status);
 
 /* Number of streaming multiprocessors the library sizes its grids for. */
 int dt_num_sms(void);
+
+/* Kernel kinds reported by the profiling hook. */
+typedef enum {
+  DT_K_BUILD_INIT = 0,
+  DT_K_MARKOV_GEMM = 1,   /* one wave of the Markov-head GEMM + fused epilogue */
+  DT_K_FRONTIER = 2,      /* one wave of the best-first frontier              */
+  DT_K_DRAFT_Q = 3,       /* draft distributions of the final tree (T > 0)    */
+  DT_K_ACCEPT_PREPASS = 4,
+  DT_K_ACCEPT_WALK = 5,
+  DT_K_ATTN = 6,
+  DT_K_ATTN_COMBINE = 7,
+  DT_K_OTHER = 8
+} dt_kernel_kind;
+
+/* Profiling hook (measurement only; off by default).  While set, every kernel
+ * the library launches from the calling host thread is bracketed by
+ * cudaEventRecord(events[2*i]) and cudaEventRecord(events[2*i+1]) on its
+ * stream, with kinds[i] = its dt_kernel_kind and i = (*count)++, as long as
+ * i < capacity.  events are cudaEvent_t handles created by the caller; all
+ * arrays are host memory owned by the caller.  Pass events = NULL to turn the
+ * hook off. */
+void dt_set_profile_events(void** events, int32_t* kinds, int capacity, int32_t* count);
 
 #ifdef __cplusplus
 }
