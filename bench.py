@@ -33,6 +33,13 @@ METRIC = "draft-tree rounds/s (build+verify+accept), V=151936 B=7 N=32; % roofli
 UNIT = "rounds/s"
 WORKLOAD_DESC = ("qwen3_4b-shaped round: V=151936, block B=7, k=4, N=32, Markov rank 256, "
                  "bf16 block logits, greedy (T=0), verify 32q/8kv d=128 prefix 2048, batch 1")
+DESCS = {
+    "qwen3_4b": WORKLOAD_DESC,
+    "qwen3_8b": ("qwen3_8b-shaped round: V=151936, block B=16, k=4, N=64, Markov rank 256, "
+                 "T=0.6 stochastic (Philox), verify 32q/8kv d=128 prefix 4096, batch 1"),
+    "load_adaptive": ("load-adaptive batch: 64 requests, B=7, V=151936, per-request budget from "
+                      "{chain, 8, 16, 32}, lambda 0.01, T=1.0, lognormal prefixes 512..8192"),
+}
 
 
 def parse():
@@ -43,6 +50,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--copies", type=int, default=4)
     p.add_argument("--no-oracle", action="store_true", help="skip the cpu_baseline leg")
+    p.add_argument("--workload", default=WORKLOAD, choices=["qwen3_4b", "qwen3_8b", "load_adaptive"])
     return p.parse_args()
 
 
@@ -112,7 +120,7 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -183,54 +191,69 @@ def run_ours(args):
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     bf = torch.bfloat16
-    w = make_workload(WORKLOAD, seed=rank)
+    w = make_workload(args.workload, seed=rank)
     V, Bk, N, r, k = w.V, w.Bk, w.Nmax, w.r, w.k
-    P = int(w.prefix_len[0])
-    q, kp, vp, kt, vt = attention_inputs(w, N + 1, 0)
-    host = dict(L=w.L, A=w.A, Bt=w.Bt, q=q[None], kp=kp, vp=vp, kt=kt[None], vt=vt[None])
+    B, temp = w.batch, w.temp
+    ldt = bf if w.logit_dtype == "bf16" else torch.float32
+    P = int(w.prefix_len.max())
+    att = [attention_inputs(w, N + 1, b) for b in range(B)]
+    host = dict(q=np.stack([a_[0] for a_ in att]), kp=np.concatenate([a_[1] for a_ in att]),
+                vp=np.concatenate([a_[2] for a_ in att]), kt=np.stack([a_[3] for a_ in att]),
+                vt=np.stack([a_[4] for a_ in att]))
+    pstart = np.concatenate([[0], np.cumsum(w.prefix_len)[:-1]]).astype(np.int64)
 
     def upload():
         c = {nm: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(bf) for nm, a in host.items()}
+        c["L"] = torch.from_numpy(w.L).to(dev).to(ldt)
+        c["A"] = torch.from_numpy(w.A).to(dev).to(bf)
+        c["Bt"] = torch.from_numpy(w.Bt).to(dev).to(bf)
         c["root"] = torch.from_numpy(w.root).to(dev)
         c["nb"] = torch.from_numpy(w.n_budget).to(dev)
+        c["kreq"] = torch.from_numpy(w.k_req).to(dev)
         c["lam"] = torch.from_numpy(w.lam).to(dev)
-        c["pstart"] = torch.zeros(1, dtype=torch.int64, device=dev)
+        c["pstart"] = torch.from_numpy(pstart).to(dev)
         c["plen"] = torch.from_numpy(w.prefix_len).to(dev)
         return c
 
     copies = [upload() for _ in range(args.copies)]
-    tree = dt.Tree.empty(1, N, device=dev)
-    ws_b = dt.workspace(dt.build_workspace_bytes(1, Bk, V, r, k, N), dev)
-    ws_v = dt.workspace(dt.verify_workspace_bytes(1, N, w.Hq, w.Hkv, w.d, P), dev)
-    ws_a = dt.workspace(dt.accept_workspace_bytes(1, N, V), dev)
-    attn_out = torch.empty(1, N + 1, w.Hq, w.d, dtype=bf, device=dev)
-    acc = torch.empty(1, Bk, dtype=torch.int32, device=dev)
-    nacc = torch.empty(1, dtype=torch.int32, device=dev)
-    bonus = torch.empty(1, dtype=torch.int32, device=dev)
+    tree = dt.Tree.empty(B, N, V, stochastic=temp > 0, device=dev)
+    ws_b = dt.workspace(dt.build_workspace_bytes(B, Bk, V, r, k, N), dev)
+    ws_v = dt.workspace(dt.verify_workspace_bytes(B, N, w.Hq, w.Hkv, w.d, P), dev)
+    ws_a = dt.workspace(dt.accept_workspace_bytes(B, N, V), dev)
+    attn_out = torch.empty(B, N + 1, w.Hq, w.d, dtype=bf, device=dev)
+    acc = torch.empty(B, Bk, dtype=torch.int32, device=dev)
+    nacc = torch.empty(B, dtype=torch.int32, device=dev)
+    bonus = torch.empty(B, dtype=torch.int32, device=dev)
     scale = 1.0 / math.sqrt(w.d)
+    seed_b, seed_a = 0x5EED, 0xACCE
 
     def build(c):
-        dt.tree_build(c["L"], c["A"], c["Bt"], c["root"], c["nb"], c["lam"], k=k, Nmax=N, temp=0.0,
-                      out=tree, ws=ws_b)
+        dt.tree_build(c["L"], c["A"], c["Bt"], c["root"], c["nb"], c["lam"], k=k, Nmax=N, temp=temp,
+                      out=tree, ws=ws_b, k_req=c["kreq"], philox_seed=seed_b)
 
     def verify(c):
         dt.tree_verify_attn(c["q"], c["kp"], c["vp"], c["pstart"], c["plen"], P, c["kt"], c["vt"],
                             tree.anc, tree.n_nodes, scale, attn_out, ws_v)
 
     def accept_(c):
-        dt.tree_accept(c["tgt"], tree, Bk, 0.0, acc, nacc, bonus, ws_a)
+        dt.tree_accept(c["tgt"], tree, Bk, temp, acc, nacc, bonus, ws_a, philox_seed=seed_a)
 
-    # the synthetic target model scores the tree this workload builds
+    # the synthetic target model scores the trees this workload builds
     build(copies[0])
     assert dt.read_status(ws_b) == 0
-    n = int(tree.n_nodes[0])
-    depths = tree.depths[0, :n].cpu().numpy()
-    tokens = tree.tokens[0, :n].cpu().numpy()
-    tgt = np.zeros((N + 1, V), np.float32)
-    tgt[: n + 1] = target_rows(w, 0, np.concatenate([[0], depths]),
-                               np.concatenate([w.root[:1], tokens]))
+    tgt = np.zeros((B, N + 1, V), np.float32)
+    n_nodes = tree.n_nodes.cpu().numpy()
+    inner = 0
+    for b in range(B):
+        n = int(n_nodes[b])
+        depths = tree.depths[b, :n].cpu().numpy()
+        tokens = tree.tokens[b, :n].cpu().numpy()
+        inner += 1 + int((depths < Bk).sum())
+        tgt[b, : n + 1] = target_rows(w, b, np.concatenate([[0], depths]),
+                                      np.concatenate([w.root[b:b + 1], tokens]))
     for c in copies:
-        c["tgt"] = torch.from_numpy(tgt[None]).to(dev).to(bf)
+        c["tgt"] = torch.from_numpy(tgt).to(dev).to(ldt)
+    n = int(n_nodes.sum())
 
     def round_(c):
         build(c)
@@ -309,27 +332,44 @@ def run_ours(args):
     kern = {nm: {"launches_per_step": len(v) / kprof, "avg_us": 1e3 * statistics.mean(v),
                  "us_per_step": 1e3 * sum(v) / kprof} for nm, v in per_kind.items()}
 
-    # ---- roofline of the dominant kernel (the Markov GEMM waves)
+    # ---- roofline of the dominant kernel (the Markov GEMM waves).  Per launch
+    # it must stream the whole Markov factor Bm [V][r] bf16 once, read the
+    # block-logit rows of the requests, the gathered node rows and write one
+    # fp32 row of scaled logits per expanded node.  `cols` = expanded nodes
+    # per wave, counted from the final trees (wasted expansions excluded).
     pk, pk_kind = peaks()
-    ncta = min(dt.num_sms(), (V + 127) // 128)
-    gemm_bytes = V * r * 2 + V * 2 + N * r * 2 + ncta * N * (8 + 8 * k)
+    cols = inner / Bk
+    lbytes = 2 if w.logit_dtype == "bf16" else 4
+    gemm_bytes = V * r * 2 + B * V * lbytes + cols * (V * 4 + r * 2)
+    gemm_flops = 2.0 * cols * V * r
     g_us = kern["markov_gemm"]["avg_us"]
-    achieved = gemm_bytes / (g_us * 1e-6) / 1e9
-    roof = {"kernel": "markov_gemm (one wave: tcgen05 GEMM + fused top-k/LSE epilogue)",
-            "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": round(achieved / pk["hbm_gbs"], 4), "peak_kind": pk_kind,
-            "algorithmic_bytes_per_launch": gemm_bytes,
-            "traffic": traffic_from_profile(os.path.join(
-                ROOT, "draft_tree_construction_markov_b200", "csrc", "markov_gemm.cu")),
-            "avg_launch_us": round(g_us, 3)}
+    t_hbm = gemm_bytes / (pk["hbm_gbs"] * 1e9)
+    t_tc = gemm_flops / (pk["bf16_tflops"] * 1e12)
+    if t_tc > t_hbm:
+        achieved = gemm_flops / (g_us * 1e-6) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        achieved = gemm_bytes / (g_us * 1e-6) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s"}
+    roof.update({"frac": round(achieved / roof["peak"], 4), "peak_kind": pk_kind,
+                 "kernel": "markov_gemm (one wave: tcgen05 Markov-head GEMM, s-row epilogue)",
+                 "algorithmic_bytes_per_launch": int(gemm_bytes),
+                 "algorithmic_flops_per_launch": int(gemm_flops),
+                 "nodes_per_wave": round(cols, 2),
+                 "traffic": traffic_from_profile(os.path.join(
+                     ROOT, "draft_tree_construction_markov_b200", "csrc", "markov_gemm.cu")),
+                 "avg_launch_us": round(g_us, 3)})
 
     # ---- end to end through the public API: pinned host inputs, copies timed
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(bf).pin_memory()
-    h_in = dict(L=pin(w.L), q=pin(q[None]), kt=pin(kt[None]), vt=pin(vt[None]), tgt=pin(tgt[None]))
+    pinl = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(ldt).pin_memory()
+    h_in = dict(L=pinl(w.L), q=pin(host["q"]), kt=pin(host["kt"]), vt=pin(host["vt"]), tgt=pinl(tgt))
     h_root = torch.from_numpy(w.root).pin_memory()
     h_out = {nm: torch.empty(sz, dtype=torch.int32).pin_memory()
-             for nm, sz in (("tok", (1, N)), ("par", (1, N)), ("n", (1,)), ("acc", (1, Bk)),
-                            ("nacc", (1,)), ("bonus", (1,)))}
+             for nm, sz in (("tok", (B, N)), ("par", (B, N)), ("n", (B,)), ("acc", (B, Bk)),
+                            ("nacc", (B,)), ("bonus", (B,)))}
     h2d = sum(t.numel() * t.element_size() for t in h_in.values()) + h_root.numel() * 4
     d2h = sum(t.numel() * t.element_size() for t in h_out.values())
     c = copies[0]
@@ -370,9 +410,10 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESC, "l2": f"inputs rotated over {args.copies} copies "
+        "config": {"workload": DESCS[args.workload], "l2": f"inputs rotated over {args.copies} copies "
                    f"({args.copies * (2 * V * r * 2) / 1e6:.0f} MB of Markov factors > 126 MB L2)",
-                   "round": "CUDA graph per input copy", "batch_per_gpu": 1,
+                   "round": "CUDA graph per input copy", "batch_per_gpu": B,
+                   "request_rounds_per_s": round(B * value, 1),
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
         "kernels": {nm: {kk: round(vv, 3) for kk, vv in d.items()} for nm, d in kern.items()},
@@ -381,8 +422,8 @@ def run_ours(args):
         "clocks": clk,
         "tree_nodes": n,
     }
-    if rank == 0 and world == 1 and not args.no_oracle:
-        v, nr, el = time_oracle(w, tgt, budget_s=20.0)
+    if rank == 0 and world == 1 and not args.no_oracle and args.workload == WORKLOAD:
+        v, nr, el = time_oracle(w, tgt[0], budget_s=20.0)
         out["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": blas_threads(),
                                "kind": "oracle",
                                "sample": f"{nr} full rounds of the same workload in {el:.1f} s "

@@ -57,7 +57,7 @@ _sig("dt_set_profile_events", None, ctypes.POINTER(ctypes.c_void_p), ctypes.POIN
      _i32, ctypes.POINTER(ctypes.c_int32))
 
 KERNEL_KINDS = ["build_init", "markov_gemm", "frontier", "draft_q", "accept_prepass",
-                "accept_walk", "attn", "attn_combine", "other"]
+                "accept_walk", "attn", "attn_combine", "topk_rows", "other"]
 
 
 class DtreeError(RuntimeError):

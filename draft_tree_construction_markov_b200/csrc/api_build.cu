@@ -15,6 +15,8 @@ cudaError_t launch_markov_gemm(int mode, bool stoch, const CUtensorMap& tmW,
 cudaError_t launch_frontier(const FrontierArgs& f, cudaStream_t s);
 cudaError_t launch_build_init(const FrontierArgs& f, const int32_t* root_token, Row* rows0,
                               int32_t* count0, cudaStream_t s);
+int topk_chunks(int Mcap, int V);
+cudaError_t launch_topk_rows(const TopkArgs& a, bool stoch, cudaStream_t s);
 
 // ------------------------------------------------------------ profile hook --
 static thread_local void** g_prof_events = nullptr;
@@ -88,13 +90,19 @@ struct BuildLayout {
   Row* mat_rows;
   uint16_t* H;
   uint16_t* Hm;
+  float* Z;  // [Mcap][V] scaled logits of the current wave
   float2* stats;
   float* lv;
   int32_t* li;
   float* gv;
   int32_t* gi;
+  int32_t* row_done;
+  float* fin_lse;
+  float* fin_v;
+  int32_t* fin_i;
+  int32_t* fin_g;
   size_t bytes;
-  int ncta_v, n_vtiles, nt, Mcap, Mcap_pad, Mmat, Mmat_pad;
+  int ncta_v, n_vtiles, nt, Mcap, Mcap_pad, Mmat, Mmat_pad, nchunk, chunk;
 };
 
 static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k, int Nmax) {
@@ -118,12 +126,20 @@ static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k
   L.mat_rows = c.take<Row>(L.Mmat);
   L.H = c.take<uint16_t>((size_t)L.Mcap_pad * r);
   L.Hm = c.take<uint16_t>((size_t)L.Mmat_pad * r);
-  const size_t np = (size_t)L.ncta_v * L.Mcap;
+  L.Z = c.take<float>((size_t)L.Mcap * V);
+  L.nchunk = topk_chunks(L.Mcap, V);
+  L.chunk = (V + L.nchunk - 1) / L.nchunk;
+  const size_t np = (size_t)L.nchunk * L.Mcap;
   L.stats = c.take<float2>(np);
   L.lv = c.take<float>(np * k);
   L.li = c.take<int32_t>(np * k);
   L.gv = c.take<float>(np * k);
   L.gi = c.take<int32_t>(np * k);
+  L.row_done = c.take<int32_t>(L.Mcap);
+  L.fin_lse = c.take<float>(L.Mcap);
+  L.fin_v = c.take<float>((size_t)L.Mcap * k);
+  L.fin_i = c.take<int32_t>((size_t)L.Mcap * k);
+  L.fin_g = c.take<int32_t>((size_t)L.Mcap * k);
   L.bytes = align_up(c.off, 256);
   return L;
 }
@@ -180,6 +196,7 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
     return DT_ECUDA;
 
   if (cudaMemsetAsync(L.status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
+  if (cudaMemsetAsync(L.row_done, 0, (size_t)L.Mcap * 4, s) != cudaSuccess) return DT_ECUDA;
 
   FrontierArgs f;
   memset(&f, 0, sizeof(f));
@@ -190,16 +207,14 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   f.A = d_markov_a;
   f.req = L.req;
   f.lists = L.lists;
-  f.stats = L.stats;
-  f.lv = L.lv;
-  f.li = L.li;
-  f.gv = L.gv;
-  f.gi = L.gi;
+  f.fin_lse = L.fin_lse;
+  f.fin_v = L.fin_v;
+  f.fin_i = L.fin_i;
+  f.fin_g = L.fin_g;
   f.calib = d_calib;
   f.n_budget = d_n_budget;
   f.k_req = d_k_req;
   f.lambda = d_lambda;
-  f.ncta_v = L.ncta_v;
   f.Mcap = L.Mcap;
   f.Bk = Bk;
   f.V = V;
@@ -225,13 +240,32 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   g.temp = temp;
   g.seed = philox_seed;
   g.offset = (uint32_t)philox_offset;
-  g.stats = L.stats;
-  g.lv = L.lv;
-  g.li = L.li;
-  g.gv = L.gv;
-  g.gi = L.gi;
+  g.out = L.Z;
   g.nmax1 = Nmax + 1;
   g.status = L.status;
+
+  TopkArgs tk;
+  memset(&tk, 0, sizeof(tk));
+  tk.S = L.Z;
+  tk.Mcap = L.Mcap;
+  tk.V = V;
+  tk.k = k;
+  tk.nchunk = L.nchunk;
+  tk.chunk = L.chunk;
+  tk.temp = temp;
+  tk.seed = philox_seed;
+  tk.offset = (uint32_t)philox_offset;
+  tk.stats = L.stats;
+  tk.lv = L.lv;
+  tk.li = L.li;
+  tk.gv = L.gv;
+  tk.gi = L.gi;
+  tk.row_done = L.row_done;
+  tk.fin_lse = L.fin_lse;
+  tk.fin_v = L.fin_v;
+  tk.fin_i = L.fin_i;
+  tk.fin_g = L.fin_g;
+  tk.status = L.status;
 
   {
     ProfileScope ps(DT_K_BUILD_INIT, s);
@@ -248,6 +282,12 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
       ProfileScope ps(DT_K_MARKOV_GEMM, s);
       if (launch_markov_gemm(EPI_EXPAND, stoch, tmW, tmH, g, batch, L.nt, s) != cudaSuccess)
         return DT_ECUDA;
+    }
+    {
+      ProfileScope ps(DT_K_TOPK, s);
+      tk.rows = L.rows[cur];
+      tk.n_rows = L.counts + cur;
+      if (launch_topk_rows(tk, stoch, s) != cudaSuccess) return DT_ECUDA;
     }
     f.rows = L.rows[cur];
     f.next_rows = L.rows[nxt];

@@ -39,6 +39,10 @@ struct ReqState {
   int32_t row_base;   // rows of this request in the current wave list
   int32_t row_count;
   float root_lse;
+  int32_t root_token;
+  float thr;          // fp32(log(lambda)), -inf for lambda = 0
+  int32_t kb;         // children per node of this request
+  int32_t nb;         // node budget of this request
   int32_t pad[2];
 };
 
@@ -57,17 +61,33 @@ struct GemmArgs {
   float temp;
   uint64_t seed;
   uint32_t offset;
-  // EPI_EXPAND partial outputs, indexed [cta_v][row]
-  float2* stats;         // (max, sum exp(s - max))
-  float* lv;             // [cta_v][row][k] top-k s values
-  int32_t* li;           // ... and their token ids
-  float* gv;             // [cta_v][row][k] top-k Gumbel keys (T > 0)
-  int32_t* gi;
-  // EPI_ZDUMP / EPI_QROWS output
-  float* out;            // zdump: [aux][V]; qrows: [b][Nmax+1][V] with row aux
+  // output rows: expand: s = z / T, [row][V]; zdump: z, [aux][V];
+  // qrows: q = exp(s - lse), [b][Nmax+1][V] with row aux
+  float* out;
   int nmax1;             // Nmax + 1
   int32_t* status;
   int stages;
+};
+
+struct TopkArgs {
+  const float* S;        // [Mcap][V] scaled logits of this wave's nodes
+  const Row* rows;
+  const int32_t* n_rows;
+  int Mcap, V, k, nchunk, chunk;
+  float temp;
+  uint64_t seed;
+  uint32_t offset;
+  float2* stats;         // [Mcap][nchunk] (max, sum exp(s - max))
+  float* lv;             // [Mcap][nchunk][k] top-k of s
+  int32_t* li;
+  float* gv;             // [Mcap][nchunk][k] Gumbel top-k (T > 0)
+  int32_t* gi;
+  int32_t* row_done;     // [Mcap] chunks finished per row (the last one merges and resets)
+  float* fin_lse;        // [Mcap] merged results per node
+  float* fin_v;          // [Mcap][k] top-k values of s (order statistics)
+  int32_t* fin_i;        // [Mcap][k] their tokens
+  int32_t* fin_g;        // [Mcap][k] Gumbel-top-k tokens (T > 0)
+  int32_t* status;
 };
 
 struct FrontierArgs {
@@ -82,16 +102,15 @@ struct FrontierArgs {
   const uint16_t* A;     // [V][r]
   ReqState* req;
   Cand* lists;           // [batch][Nmax]
-  const float2* stats;
-  const float* lv;
-  const int32_t* li;
-  const float* gv;
-  const int32_t* gi;
+  const float* fin_lse;  // [Mcap] per expanded node: log-sum-exp of s
+  const float* fin_v;    // [Mcap][k] top-k values of s
+  const int32_t* fin_i;  // [Mcap][k] their tokens
+  const int32_t* fin_g;  // [Mcap][k] Gumbel-top-k tokens (T > 0)
   const float* calib;    // [Bk][2] or NULL
   const int32_t* n_budget;
   const int32_t* k_req;
   const float* lambda;
-  int ncta_v, Mcap, Bk, V, r, k, Nmax, batch;
+  int Mcap, Bk, V, r, k, Nmax, batch;
   float temp;
   dt_tree out;
   int32_t* status;

@@ -64,6 +64,21 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
                : "r"(addr));
 }
 
+// 16-byte global -> shared copy that does not block the thread; zero-fills
+// the destination when `pred` is false.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool pred) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(pred ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Is tree column j (0 = root, j' + 1 = node j') visible from tree row i?
 __device__ __forceinline__ bool tree_visible(int i, int j, uint64_t anc_row) {
   return j == 0 || (i >= 1 && ((anc_row >> (j - 1)) & 1ull));
@@ -74,8 +89,7 @@ __global__ void __launch_bounds__(512) attn_bf16_kernel(AttnArgs a) {
   constexpr int LD = D + 8;  // padded row (bf16 elements) against bank conflicts
   extern __shared__ __align__(16) uint8_t asmem[];
   uint16_t* sQ = (uint16_t*)asmem;                 // [rows_per_cta][LD]
-  uint16_t* sK = sQ + (size_t)a.rows_per_cta * LD; // [kChunk][LD]
-  uint16_t* sV = sK + kChunk * LD;                 // [kChunk][LD]
+  uint16_t* sKV = sQ + (size_t)a.rows_per_cta * LD; // 2 x ([kChunk][LD] K, [kChunk][LD] V)
   const int split = blockIdx.x, kvh = blockIdx.y;
   const int b = blockIdx.z / a.n_rblocks, rb = blockIdx.z % a.n_rblocks;
   const int n = min(max(a.n_nodes[b], 0), a.Nmax);
@@ -97,12 +111,10 @@ __global__ void __launch_bounds__(512) attn_bf16_kernel(AttnArgs a) {
   for (int idx = tid; idx < a.rows_per_cta * (D / 8); idx += nthreads) {
     const int rr = idx / (D / 8), cc = idx % (D / 8);
     const int rho = row0 + rr;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (rho < R) {
-      const int i = rho / a.G, hh = rho % a.G;
-      v = *(const uint4*)(q + (((size_t)b * (a.Nmax + 1) + i) * a.Hq + kvh * a.G + hh) * D + cc * 8);
-    }
-    *(uint4*)(sQ + (size_t)rr * LD + cc * 8) = v;
+    const bool ok = rho < R;
+    const int i = ok ? rho / a.G : 0, hh = ok ? rho % a.G : 0;
+    cp_async16(sQ + (size_t)rr * LD + cc * 8,
+               q + (((size_t)b * (a.Nmax + 1) + i) * a.Hq + kvh * a.G + hh) * D + cc * 8, ok);
   }
   // per-lane rows (g and g + 8 of the warp's 16-row tile)
   const int g = lane >> 2, t4 = lane & 3;
@@ -126,32 +138,44 @@ __global__ void __launch_bounds__(512) attn_bf16_kernel(AttnArgs a) {
   const uint16_t* vtr = (const uint16_t*)a.vt;
   const int64_t ps = a.pstart[b];
 
-  for (int cb = c0; cb < c1; cb += kChunk) {
-    __syncthreads();
+  // K/V chunk loader: buffer `buf` <- columns [cb, cb + kChunk)
+  auto load_chunk = [&](int cb, int buf) {
+    uint16_t* dK = sKV + (size_t)buf * 2 * kChunk * LD;
+    uint16_t* dV = dK + kChunk * LD;
     for (int idx = tid; idx < kChunk * (D / 8); idx += nthreads) {
       const int rr = idx / (D / 8), cc = idx % (D / 8);
       const int c = cb + rr;
-      uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-      if (c < c1) {
-        size_t off;
-        const uint16_t *ks, *vs;
-        if (c < P) {
-          off = ((size_t)(ps + c) * a.Hkv + kvh) * D + cc * 8;
-          ks = kp;
-          vs = vp;
-        } else {
-          off = (((size_t)b * (a.Nmax + 1) + (c - P)) * a.Hkv + kvh) * D + cc * 8;
-          ks = ktr;
-          vs = vtr;
-        }
-        kv = *(const uint4*)(ks + off);
-        vv = *(const uint4*)(vs + off);
+      const bool ok = c < c1;
+      size_t off;
+      const uint16_t *ks, *vs;
+      if (!ok) {  // zero-filled; the source is any valid address
+        off = 0;
+        ks = ktr;
+        vs = vtr;
+      } else if (c < P) {
+        off = ((size_t)(ps + c) * a.Hkv + kvh) * D + cc * 8;
+        ks = kp;
+        vs = vp;
+      } else {
+        off = (((size_t)b * (a.Nmax + 1) + (c - P)) * a.Hkv + kvh) * D + cc * 8;
+        ks = ktr;
+        vs = vtr;
       }
-      *(uint4*)(sK + (size_t)rr * LD + cc * 8) = kv;
-      *(uint4*)(sV + (size_t)rr * LD + cc * 8) = vv;
+      cp_async16(dK + (size_t)rr * LD + cc * 8, ks + off, ok);
+      cp_async16(dV + (size_t)rr * LD + cc * 8, vs + off, ok);
     }
+  };
+  if (c0 < c1) load_chunk(c0, 0);
+  cp_async_commit();  // group: Q + first chunk
+  int buf = 0;
+  for (int cb = c0; cb < c1; cb += kChunk, buf ^= 1) {
+    if (cb + kChunk < c1) load_chunk(cb + kChunk, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();  // everything but the chunk just issued has landed
     __syncthreads();
-    if (!warp_active) continue;
+    const uint16_t* sK = sKV + (size_t)buf * 2 * kChunk * LD;
+    const uint16_t* sV = sK + kChunk * LD;
+    if (warp_active) {
     // S = Q K^T for 16 rows x 64 columns
     float s[kChunk / 8][4];
 #pragma unroll
@@ -235,7 +259,10 @@ __global__ void __launch_bounds__(512) attn_bf16_kernel(AttnArgs a) {
         mma_bf16_16816(o[nt + 1], af, bf[2], bf[3]);
       }
     }
+    }  // warp_active
+    __syncthreads();  // buffer `buf` is refilled by the next iteration's loads
   }
+  cp_async_wait<0>();
   if (!warp_active) return;
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
@@ -258,14 +285,16 @@ __global__ void __launch_bounds__(512) attn_bf16_kernel(AttnArgs a) {
 }
 
 constexpr int kMaxSplits = 512;
+constexpr int kCombineWarps = 4;
 
-// Merge the column splits: grid (batch * (Nmax+1), Hq), 128 threads.
+// Merge the column splits: one warp per (request, row, head); lanes cover
+// head_dim in 4-float vectors.  grid (ceil(batch*(Nmax+1)*Hq / 4)), 128 threads.
 __global__ void attn_combine_kernel(AttnArgs a) {
-  __shared__ float s_w[kMaxSplits];
-  __shared__ float s_l[kMaxSplits];
-  __shared__ float s_red[2];
-  const int b = blockIdx.x / (a.Nmax + 1), i = blockIdx.x % (a.Nmax + 1);
-  const int h = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int item = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  const int per_b = (a.Nmax + 1) * a.Hq;
+  if (item >= a.batch * per_b) return;
+  const int b = item / per_b, i = (item % per_b) / a.Hq, h = item % a.Hq;
   if (i > min(a.n_nodes[b], a.Nmax)) return;
   const int kvh = h / a.G, hh = h % a.G;
   const int rho = i * a.G + hh;
@@ -276,35 +305,39 @@ __global__ void attn_combine_kernel(AttnArgs a) {
   const size_t split_stride = (size_t)a.batch * a.Hkv * a.n_rblocks * a.rpad;
   const size_t pb0 = ((size_t)b * a.Hkv + kvh) * (size_t)(a.n_rblocks * a.rpad) +
                      rb * a.rows_per_cta + rl;
-  for (int s = threadIdx.x; s < used; s += blockDim.x) {
+  float mx = -INFINITY;
+  for (int s = lane; s < used; s += 32) mx = fmaxf(mx, a.part_ml[pb0 + s * split_stride].x);
+  mx = warp_max(mx);
+  float l = 0.f;
+  for (int s = lane; s < used; s += 32) {
     const float2 ml = a.part_ml[pb0 + s * split_stride];
-    s_w[s] = ml.x;
-    s_l[s] = ml.y;
+    if (ml.x != -INFINITY) l += exp2f(ml.x - mx) * ml.y;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float mx = -INFINITY;
-    for (int s = 0; s < used; ++s) mx = fmaxf(mx, s_w[s]);
-    float l = 0.f;
+  l = warp_sum(l);
+  const float inv_l = 1.f / l;
+  const int nvec = a.d / 4;  // 16 or 32 float4 per row
+  if (lane < nvec) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
     for (int s = 0; s < used; ++s) {
-      const float wgt = s_w[s] == -INFINITY ? 0.f : exp2f(s_w[s] - mx);
-      s_w[s] = wgt;
-      l += wgt * s_l[s];
+      const float2 ml = a.part_ml[pb0 + s * split_stride];
+      const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - mx);
+      const float4 o = ((const float4*)(a.part_o + (pb0 + s * split_stride) * a.d))[lane];
+      acc.x += w * o.x;
+      acc.y += w * o.y;
+      acc.z += w * o.z;
+      acc.w += w * o.w;
     }
-    s_red[0] = l;
-  }
-  __syncthreads();
-  const float inv_l = 1.f / s_red[0];
-  for (int dd = threadIdx.x; dd < a.d; dd += blockDim.x) {
-    float acc = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < used; ++s) acc += s_w[s] * a.part_o[(pb0 + s * split_stride) * a.d + dd];
-    const float v = acc * inv_l;
-    const size_t oi = (((size_t)b * (a.Nmax + 1) + i) * a.Hq + h) * a.d + dd;
-    if (a.out_bf16)
-      ((uint16_t*)a.out)[oi] = (uint16_t)(pack_bf16(v, 0.f) & 0xFFFF);
-    else
-      ((float*)a.out)[oi] = v;
+    const size_t oi = (((size_t)b * (a.Nmax + 1) + i) * a.Hq + h) * a.d + 4 * lane;
+    if (a.out_bf16) {
+      uint2 pk;
+      pk.x = pack_bf16(acc.x * inv_l, acc.y * inv_l);
+      pk.y = pack_bf16(acc.z * inv_l, acc.w * inv_l);
+      *(uint2*)((uint16_t*)a.out + oi) = pk;
+    } else {
+      *(float4*)((float*)a.out + oi) =
+          make_float4(acc.x * inv_l, acc.y * inv_l, acc.z * inv_l, acc.w * inv_l);
+    }
   }
 }
 
@@ -398,7 +431,7 @@ static AttnPlan attn_plan(int batch, int Nmax, int Hq, int Hkv, int d, int max_p
   const int Cmax = max_prefix + Nmax + 1;
   const int chunks = (Cmax + kChunk - 1) / kChunk;
   const int base_ctas = batch * Hkv * p.n_rblocks;
-  int want = (2 * 148 + base_ctas - 1) / base_ctas;
+  int want = (148 + base_ctas - 1) / base_ctas;
   want = std::max(1, std::min(want, chunks));
   const int chunks_per = (chunks + want - 1) / want;
   p.cols_per_split = chunks_per * kChunk;
@@ -481,7 +514,7 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const voi
     attn_f32_kernel<<<dim3(batch * (Nmax + 1), Hq), 128, smem, s>>>(a, max_cols);
     return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ECUDA;
   }
-  const size_t smem = ((size_t)p.rows_per_cta + 2 * kChunk) * (d + 8) * 2;
+  const size_t smem = ((size_t)p.rows_per_cta + 4 * kChunk) * (d + 8) * 2;
   dim3 grid(p.splits, Hkv, batch * p.n_rblocks);
   const int threads = 32 * std::max(p.warps, 4);
   {
@@ -498,7 +531,8 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const voi
   if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
   }
   ProfileScope ps(DT_K_ATTN_COMBINE, s);
-  attn_combine_kernel<<<dim3(batch * (Nmax + 1), Hq), 128, 0, s>>>(a);
+  const int items = batch * (Nmax + 1) * Hq;
+  attn_combine_kernel<<<(items + kCombineWarps - 1) / kCombineWarps, 32 * kCombineWarps, 0, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ECUDA;
 }
 

@@ -196,7 +196,8 @@ typedef enum {
   DT_K_ACCEPT_WALK = 5,
   DT_K_ATTN = 6,
   DT_K_ATTN_COMBINE = 7,
-  DT_K_OTHER = 8
+  DT_K_TOPK = 8,          /* one wave of softmax statistics + top-k per node  */
+  DT_K_OTHER = 9
 } dt_kernel_kind;
 
 /* Profiling hook (measurement only; off by default).  While set, every kernel
