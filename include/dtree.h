@@ -178,6 +178,34 @@ dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt,
                          int32_t* d_n_acc, int32_t* d_bonus, void* ws,
                          size_t ws_bytes, dt_stream stream);
 
+/* dt_tree_accept for callers that cannot allocate device memory.  The pages
+ * have no counterpart of this entry point; it is a deployment convenience.
+ * Some callers cannot hand the library a workspace: a plugin running inside a
+ * host framework whose caching allocator owns the device's memory and offers
+ * it no allocation hook, or a latency-critical serving loop that must never
+ * call cudaMalloc (it may synchronise the device and its latency is
+ * unbounded).  This variant takes the same arguments as dt_tree_accept
+ * without `ws`/`ws_bytes`; its scratch is a fixed 2 MiB array in the library's
+ * device memory, which every GPU that loads the library holds until the
+ * process exits.  It allocates nothing and frees nothing.
+ *   - Supported sizes: dt_tree_accept_workspace_bytes(batch, Nmax, V) <= 2 MiB
+ *     (e.g. batch 1 at V = 151936); larger sizes return DT_EUNSUPPORTED with
+ *     nothing enqueued.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     temporaries; calls that overlap on the GPU race, so serialise them
+ *     (e.g. one stream).  Outputs are written to the caller's buffers only.
+ *   - Device-side range failures of this variant are not reported through a
+ *     readable status word. */
+dt_status dt_tree_accept_noalloc(const void* d_target_logits, dt_dtype tdt,
+                                 const dt_tree* tree, int batch, int Bk, int V,
+                                 int Nmax, float temp, uint64_t philox_seed,
+                                 uint64_t philox_offset, int32_t* d_acc_nodes,
+                                 int32_t* d_n_acc, int32_t* d_bonus,
+                                 dt_stream stream);
+
 /* Synchronises `stream` and returns the status word that device code of the
  * last call using `ws` wrote (DT_OK, DT_ETIMEOUT or DT_EDEVICE), then clears
  * it.  `ws` is the workspace passed to that call. */
