@@ -27,6 +27,10 @@ Readings fixed here:
     rank asc).  Candidates are the top-M children of a node; a node whose
     token is outside S_depth has no evaluated distribution and is a leaf.
   * temperature 0: tokens by top-M of the logits, survival from T = 1.
+  * `store` (optional) is applied where a bf16 network stores an activation
+    that feeds the next GEMM: x, silu(g) * u and h'.  With store=bf16_rne the
+    oracle takes its top-M decisions on the same bf16 activations as a bf16
+    kernel; store=None is the plain fp64 definition.
 """
 from __future__ import annotations
 
@@ -48,12 +52,21 @@ def silu(x):
     return x / (1.0 + np.exp(-x))
 
 
-def ar_approximator(h, e_prev, w_norm_h, w_norm_e, W_gate, W_up, W_down):
+def bf16_rne(x):
+    """Round to float32, then to bfloat16 (round to nearest, ties to even); fp64 out."""
+    u = np.asarray(x, np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def ar_approximator(h, e_prev, w_norm_h, w_norm_e, W_gate, W_up, W_down, store=None):
     """h' = h + W_down(silu(W_gate x) * (W_up x)), x = [rms(h) :: rms(e_prev)]."""
-    x = np.concatenate([rmsnorm(h, w_norm_h), rmsnorm(e_prev, w_norm_e)], axis=-1)
+    keep = store if store is not None else (lambda v: v)
+    x = keep(np.concatenate([rmsnorm(h, w_norm_h), rmsnorm(e_prev, w_norm_e)], axis=-1))
     g = np.asarray(W_gate, np.float64) @ x
     u = np.asarray(W_up, np.float64) @ x
-    return np.asarray(h, np.float64) + np.asarray(W_down, np.float64) @ (silu(g) * u)
+    act = keep(silu(g) * u)
+    return keep(np.asarray(h, np.float64) + np.asarray(W_down, np.float64) @ act)
 
 
 def stage1_sets(h, W_lm, M):
@@ -62,22 +75,25 @@ def stage1_sets(h, W_lm, M):
     return [top_k_desc(W @ np.asarray(h[i], np.float64), M) for i in range(len(h))]
 
 
-def stage2_distributions(h, E, root, sets, w_norm_h, w_norm_e, W_gate, W_up, W_down, W_lm):
+def stage2_distributions(h, E, root, sets, w_norm_h, w_norm_e, W_gate, W_up, W_down, W_lm,
+                         store=None):
     """{(depth, prev): (s, lse)} for depth 1 (prev = root) and every prev in S_{depth-1}."""
     W = np.asarray(W_lm, np.float64)
     out = {}
     evals = [(1, int(root))] + [(i, int(t)) for i in range(2, len(h) + 1) for t in sets[i - 2]]
     for d, prev in evals:
-        hp = ar_approximator(h[d - 1], E[prev], w_norm_h, w_norm_e, W_gate, W_up, W_down)
+        hp = ar_approximator(h[d - 1], E[prev], w_norm_h, w_norm_e, W_gate, W_up, W_down, store)
         out[(d, prev)] = scaled_logits(W @ hp, 0.0)
     return out
 
 
-def treeflash_tree(h, E, root, M, budget, w_norm_h, w_norm_e, W_gate, W_up, W_down, W_lm):
+def treeflash_tree(h, E, root, M, budget, w_norm_h, w_norm_e, W_gate, W_up, W_down, W_lm,
+                   store=None):
     """Best-first top-`budget` tree over the stage-2 distributions of one request."""
     gamma = len(h)
     sets = stage1_sets(h, W_lm, M)
-    dist = stage2_distributions(h, E, root, sets, w_norm_h, w_norm_e, W_gate, W_up, W_down, W_lm)
+    dist = stage2_distributions(h, E, root, sets, w_norm_h, w_norm_e, W_gate, W_up, W_down, W_lm,
+                                store)
     in_set = [set(int(t) for t in s) for s in sets]
 
     heap = []

@@ -108,3 +108,25 @@ def test_tree_is_brute_force_top_b(seed, M, B):
             node = tree.parents[node]
         got.add(tuple(reversed(path)))
     assert got == want
+
+
+def test_bf16_store_matches_torch_rounding():
+    """bf16_rne is round-to-nearest-even on the fp32 value (torch's bfloat16 cast)."""
+    g = np.random.default_rng(7)
+    x = np.concatenate([g.standard_normal(4000) * 10.0 ** g.integers(-3, 4, 4000),
+                        # exact halfway cases between two bf16 neighbours
+                        (np.arange(1, 200, dtype=np.float64) * 2 + 1) * 2.0 ** -8])
+    want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(treeflash.bf16_rne(x), want)
+
+
+def test_bf16_store_stays_within_bf16_error():
+    x = _inputs(8, D=16, Dff=16)
+    plain = treeflash.ar_approximator(x["h"][0], x["E"][2], x["w_norm_h"], x["w_norm_e"],
+                                      x["W_gate"], x["W_up"], x["W_down"])
+    stored = treeflash.ar_approximator(x["h"][0], x["E"][2], x["w_norm_h"], x["w_norm_e"],
+                                       x["W_gate"], x["W_up"], x["W_down"],
+                                       store=treeflash.bf16_rne)
+    assert np.all(treeflash.bf16_rne(stored) == stored)  # h' itself is stored in bf16
+    assert np.max(np.abs(stored - plain)) <= 0.05 * np.max(np.abs(plain))
+    assert not np.array_equal(stored, plain)
