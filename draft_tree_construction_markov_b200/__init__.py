@@ -118,6 +118,25 @@ def tree_accept(target_logits, tree: Tree, Bk, temp, acc_nodes, n_acc, bonus, ws
     return acc_nodes, n_acc, bonus
 
 
+def treeflash_workspace_bytes(batch, gamma, D, Dff, V, M, budget) -> int:
+    return int(_lib.lib.dt_treeflash_workspace_bytes(batch, gamma, D, Dff, V, M, budget))
+
+
+def treeflash_build(h, embed, w_norm_h, w_norm_e, w_gate, w_up, w_down, w_lm, root, *, M,
+                    budget, out: Tree, ws, stream=None):
+    """dt_treeflash_build.  h [batch,gamma,D] bf16; embed/w_lm [V,D] bf16; w_gate/w_up
+    [Dff,2D] bf16; w_down [D,Dff] bf16; w_norm_h/w_norm_e [D] fp32; root [batch] int32."""
+    batch, gamma, D = h.shape
+    V = w_lm.shape[0]
+    Dff = w_gate.shape[0]
+    st = out.c_struct()
+    check(_lib.lib.dt_treeflash_build(
+        ptr(h), ptr(embed), ptr(w_norm_h), ptr(w_norm_e), ptr(w_gate), ptr(w_up), ptr(w_down),
+        ptr(w_lm), ptr(root), batch, gamma, D, Dff, V, M, budget, ctypes.byref(st), ptr(ws),
+        ws.numel(), stream_ptr(stream)), "dt_treeflash_build")
+    return out
+
+
 def read_status(ws, stream=None) -> int:
     """Synchronise and return (then clear) the device status word of a workspace."""
     v = ctypes.c_int32(0)

@@ -20,7 +20,7 @@ DT_F32, DT_BF16 = 0, 1
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build it with "
-        "`python -m draft_tree_construction_markov_b200.build` (nvcc, sm_100a)")
+        "`python draft_tree_construction_markov_b200/build.py` (nvcc, sm_100a)")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -52,12 +52,15 @@ _sig("dt_tree_verify_attn", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, 
 _sig("dt_tree_accept_workspace_bytes", _sz, _i32, _i32, _i32)
 _sig("dt_tree_accept", _i32, _vp, _i32, ctypes.POINTER(DtTree), _i32, _i32, _i32, _i32, _f32,
      _u64, _u64, _vp, _vp, _vp, _vp, _sz, _vp)
+_sig("dt_treeflash_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32, _i32)
+_sig("dt_treeflash_build", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+     _i32, _i32, _i32, _i32, ctypes.POINTER(DtTree), _vp, _sz, _vp)
 _sig("dt_read_status", _i32, _vp, _vp, ctypes.POINTER(ctypes.c_int32))
 _sig("dt_set_profile_events", None, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int32),
      _i32, ctypes.POINTER(ctypes.c_int32))
 
 KERNEL_KINDS = ["build_init", "markov_gemm", "frontier", "draft_q", "accept_prepass",
-                "accept_walk", "attn", "attn_combine", "topk_rows", "other"]
+                "accept_walk", "attn", "attn_combine", "other", "tf_lmhead", "tf_mlp"]
 
 
 class DtreeError(RuntimeError):

@@ -1,6 +1,6 @@
 """Compile libdtree.so (sm_100a) in-tree with nvcc.
 
-    python -m draft_tree_construction_markov_b200.build [--verbose]
+    python draft_tree_construction_markov_b200/build.py [--verbose]
 
 The shared library lands next to this file so that it travels with the
 repository; nothing is installed into site-packages.
@@ -13,8 +13,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdtree.so")
-SOURCES = ["api_build.cu", "markov_gemm.cu", "topk_rows.cu", "frontier.cu", "accept.cu",
-           "verify_attn.cu", "accept_noalloc.cu"]
+SOURCES = ["api_build.cu", "markov_gemm.cu", "frontier.cu", "accept.cu", "verify_attn.cu",
+           "treeflash.cu", "accept_noalloc.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -10,13 +10,11 @@ bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t K, uint6
                            uint32_t box_rows);
 int gemm_node_tile(int max_cols);
 cudaError_t launch_markov_gemm(int mode, bool stoch, const CUtensorMap& tmW,
-                               const CUtensorMap& tmH, const GemmArgs& a, int batch, int nt,
-                               cudaStream_t s);
+                               const CUtensorMap& tmW2, const CUtensorMap& tmH, GemmArgs a,
+                               int batch, int nt, cudaStream_t s);
 cudaError_t launch_frontier(const FrontierArgs& f, cudaStream_t s);
 cudaError_t launch_build_init(const FrontierArgs& f, const int32_t* root_token, Row* rows0,
                               int32_t* count0, cudaStream_t s);
-int topk_chunks(int Mcap, int V);
-cudaError_t launch_topk_rows(const TopkArgs& a, bool stoch, cudaStream_t s);
 
 // ------------------------------------------------------------ profile hook --
 static thread_local void** g_prof_events = nullptr;
@@ -58,6 +56,12 @@ cudaError_t ensure_smem_ptr(const void* kernel, size_t bytes) {
   return cudaSuccess;
 }
 
+// Rows of the block logits start on 16-byte boundaries (vector bias loads).
+static int l_vec_ok(const void* L, dt_dtype ldt, int V) {
+  if ((uintptr_t)L & 15) return 0;
+  return ldt == DT_BF16 ? (V % 8 == 0) : (V % 4 == 0);
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -90,19 +94,13 @@ struct BuildLayout {
   Row* mat_rows;
   uint16_t* H;
   uint16_t* Hm;
-  float* Z;  // [Mcap][V] scaled logits of the current wave
-  float2* stats;
-  float* lv;
-  int32_t* li;
-  float* gv;
-  int32_t* gi;
-  int32_t* row_done;
-  float* fin_lse;
-  float* fin_v;
-  int32_t* fin_i;
-  int32_t* fin_g;
+  float2* pstats;  // [Mcap][ncta_v] per-CTA partials of the wave GEMM
+  float* plv;      // [Mcap][ncta_v][k]
+  int32_t* pli;
+  float* pgv;
+  int32_t* pgi;
   size_t bytes;
-  int ncta_v, n_vtiles, nt, Mcap, Mcap_pad, Mmat, Mmat_pad, nchunk, chunk;
+  int ncta_v, n_vtiles, nt, Mcap, Mcap_pad, Mmat, Mmat_pad;
 };
 
 static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k, int Nmax) {
@@ -126,20 +124,12 @@ static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k
   L.mat_rows = c.take<Row>(L.Mmat);
   L.H = c.take<uint16_t>((size_t)L.Mcap_pad * r);
   L.Hm = c.take<uint16_t>((size_t)L.Mmat_pad * r);
-  L.Z = c.take<float>((size_t)L.Mcap * V);
-  L.nchunk = topk_chunks(L.Mcap, V);
-  L.chunk = (V + L.nchunk - 1) / L.nchunk;
-  const size_t np = (size_t)L.nchunk * L.Mcap;
-  L.stats = c.take<float2>(np);
-  L.lv = c.take<float>(np * k);
-  L.li = c.take<int32_t>(np * k);
-  L.gv = c.take<float>(np * k);
-  L.gi = c.take<int32_t>(np * k);
-  L.row_done = c.take<int32_t>(L.Mcap);
-  L.fin_lse = c.take<float>(L.Mcap);
-  L.fin_v = c.take<float>((size_t)L.Mcap * k);
-  L.fin_i = c.take<int32_t>((size_t)L.Mcap * k);
-  L.fin_g = c.take<int32_t>((size_t)L.Mcap * k);
+  const size_t np = (size_t)L.ncta_v * L.Mcap;
+  L.pstats = c.take<float2>(np);
+  L.plv = c.take<float>(np * k);
+  L.pli = c.take<int32_t>(np * k);
+  L.pgv = c.take<float>(np * k);
+  L.pgi = c.take<int32_t>(np * k);
   L.bytes = align_up(c.off, 256);
   return L;
 }
@@ -196,7 +186,6 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
     return DT_ECUDA;
 
   if (cudaMemsetAsync(L.status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
-  if (cudaMemsetAsync(L.row_done, 0, (size_t)L.Mcap * 4, s) != cudaSuccess) return DT_ECUDA;
 
   FrontierArgs f;
   memset(&f, 0, sizeof(f));
@@ -207,10 +196,12 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   f.A = d_markov_a;
   f.req = L.req;
   f.lists = L.lists;
-  f.fin_lse = L.fin_lse;
-  f.fin_v = L.fin_v;
-  f.fin_i = L.fin_i;
-  f.fin_g = L.fin_g;
+  f.pstats = L.pstats;
+  f.plv = L.plv;
+  f.pli = L.pli;
+  f.pgv = L.pgv;
+  f.pgi = L.pgi;
+  f.ncta = L.ncta_v;
   f.calib = d_calib;
   f.n_budget = d_n_budget;
   f.k_req = d_k_req;
@@ -230,6 +221,7 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   memset(&g, 0, sizeof(g));
   g.L = d_block_logits;
   g.l_bf16 = ldt == DT_BF16;
+  g.l_vec = l_vec_ok(d_block_logits, ldt, V);
   g.Bk = Bk;
   g.V = V;
   g.r = r;
@@ -240,32 +232,14 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   g.temp = temp;
   g.seed = philox_seed;
   g.offset = (uint32_t)philox_offset;
-  g.out = L.Z;
+  g.pstats = L.pstats;
+  g.plv = L.plv;
+  g.pli = L.pli;
+  g.pgv = L.pgv;
+  g.pgi = L.pgi;
   g.nmax1 = Nmax + 1;
   g.status = L.status;
 
-  TopkArgs tk;
-  memset(&tk, 0, sizeof(tk));
-  tk.S = L.Z;
-  tk.Mcap = L.Mcap;
-  tk.V = V;
-  tk.k = k;
-  tk.nchunk = L.nchunk;
-  tk.chunk = L.chunk;
-  tk.temp = temp;
-  tk.seed = philox_seed;
-  tk.offset = (uint32_t)philox_offset;
-  tk.stats = L.stats;
-  tk.lv = L.lv;
-  tk.li = L.li;
-  tk.gv = L.gv;
-  tk.gi = L.gi;
-  tk.row_done = L.row_done;
-  tk.fin_lse = L.fin_lse;
-  tk.fin_v = L.fin_v;
-  tk.fin_i = L.fin_i;
-  tk.fin_g = L.fin_g;
-  tk.status = L.status;
 
   {
     ProfileScope ps(DT_K_BUILD_INIT, s);
@@ -280,14 +254,8 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
     g.reset_count = L.counts + nxt;
     {
       ProfileScope ps(DT_K_MARKOV_GEMM, s);
-      if (launch_markov_gemm(EPI_EXPAND, stoch, tmW, tmH, g, batch, L.nt, s) != cudaSuccess)
+      if (launch_markov_gemm(EPI_EXPAND, stoch, tmW, tmW, tmH, g, batch, L.nt, s) != cudaSuccess)
         return DT_ECUDA;
-    }
-    {
-      ProfileScope ps(DT_K_TOPK, s);
-      tk.rows = L.rows[cur];
-      tk.n_rows = L.counts + cur;
-      if (launch_topk_rows(tk, stoch, s) != cudaSuccess) return DT_ECUDA;
     }
     f.rows = L.rows[cur];
     f.next_rows = L.rows[nxt];
@@ -305,7 +273,7 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
     gq.Mcap = L.Mmat;
     gq.out = out->d_draft_q;
     ProfileScope ps(DT_K_DRAFT_Q, s);
-    if (launch_markov_gemm(EPI_QROWS, true, tmW, tmHm, gq, batch, L.nt, s) != cudaSuccess)
+    if (launch_markov_gemm(EPI_QROWS, true, tmW, tmW, tmHm, gq, batch, L.nt, s) != cudaSuccess)
       return DT_ECUDA;
   }
   return DT_OK;
@@ -313,26 +281,32 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
 
 // ---------------------------------------------------------------- z rows --
 namespace {
+// One warp per row: the row descriptor and the gathered Markov row A[token]
+// (r is a multiple of 16, so rows move in 16-byte pieces).
 __global__ void zrows_prep_kernel(const int32_t* req, const int32_t* depth, const int32_t* token,
-                                  int n, int V, int r, const uint16_t* A, Row* rows, uint16_t* H,
-                                  int32_t* count, int32_t* status) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
-    Row rw;
-    rw.b = req[i];
-    rw.depth = depth[i];
+                                  int n, int V, int r, const uint16_t* __restrict__ A, Row* rows,
+                                  uint16_t* __restrict__ H, int32_t* count, int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n; i += gridDim.x * wpb) {
     int t = token[i];
-    if (t < 0 || t >= V) {
-      set_status(status, DT_EDEVICE);
-      t = 0;
-      rw.b = -1;
+    const bool bad = t < 0 || t >= V;
+    if (bad) t = 0;
+    if (lane == 0) {
+      Row rw;
+      rw.b = bad ? -1 : req[i];
+      rw.depth = depth[i];
+      if (bad) set_status(status, DT_EDEVICE);
+      rw.token = t;
+      rw.aux = i;
+      rw.path = 0;
+      rw.lse = 0.f;
+      rw.key = 0.f;
+      rows[i] = rw;
     }
-    rw.token = t;
-    rw.aux = i;
-    rw.path = 0;
-    rw.lse = 0.f;
-    rw.key = 0.f;
-    rows[i] = rw;
-    for (int j = 0; j < r; ++j) H[(size_t)i * r + j] = A[(size_t)t * r + j];
+    const uint4* src = (const uint4*)(A + (size_t)t * r);
+    uint4* dst = (uint4*)(H + (size_t)i * r);
+    for (int j = lane; j < r / 8; j += 32) dst[j] = src[j];
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) *count = n;
 }
@@ -371,7 +345,7 @@ dt_status dt_markov_logits(const void* d_block_logits, dt_dtype ldt, const uint1
       !make_tmap_bf16_kmajor(&tmH, H, r, n_pad, nt))
     return DT_ECUDA;
   if (cudaMemsetAsync(hdr, 0, 4, s) != cudaSuccess) return DT_ECUDA;
-  zrows_prep_kernel<<<(n_rows + 127) / 128, 128, 0, s>>>(d_req, d_depth, d_token, n_rows, V, r,
+  zrows_prep_kernel<<<(n_rows + 7) / 8, 256, 0, s>>>(d_req, d_depth, d_token, n_rows, V, r,
                                                           d_markov_a, rows, H, hdr + 4, hdr);
   if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
   GemmArgs g;
@@ -389,7 +363,7 @@ dt_status dt_markov_logits(const void* d_block_logits, dt_dtype ldt, const uint1
   g.Mcap = n_rows;
   g.out = d_z;
   g.status = hdr;
-  if (launch_markov_gemm(EPI_ZDUMP, false, tmW, tmH, g, batch, nt, s) != cudaSuccess)
+  if (launch_markov_gemm(EPI_ZDUMP, false, tmW, tmW, tmH, g, batch, nt, s) != cudaSuccess)
     return DT_ECUDA;
   return DT_OK;
 }

@@ -46,48 +46,37 @@ struct ReqState {
   int32_t pad[2];
 };
 
-enum EpiMode { EPI_EXPAND = 0, EPI_ZDUMP = 1, EPI_QROWS = 2 };
+enum EpiMode { EPI_EXPAND = 0, EPI_ZDUMP = 1, EPI_QROWS = 2, EPI_SWIGLU = 3 };
 
 struct GemmArgs {
-  const void* L;         // block logits [batch][Bk][V]
+  const void* L;         // bias rows [batch][Bk][V] (block logits, residual) or NULL
   int l_bf16;
-  int Bk, V, r, k;
+  int l_vec;             // rows of L are 16-byte aligned (vector bias loads)
+  int Bk, V, r, k;       // V: weight rows (vocabulary / features), r: inner dimension
   const Row* rows;       // GEMM columns
   const int32_t* n_rows; // device count of valid columns
   int32_t* reset_count;  // set to 0 by CTA (0,0) (next wave's counter), may be NULL
-  int n_vtiles;          // vocab tiles of 128 rows
-  int ncta_v;            // CTAs along the vocabulary
+  int n_vtiles;          // weight tiles (128 rows; SwiGLU: 64 features)
+  int ncta_v;            // weight ranges (= partials per node)
+  int n_ntiles;          // node tiles for Mcap columns (set by the launcher)
   int Mcap;              // capacity of rows
   float temp;
   uint64_t seed;
   uint32_t offset;
-  // output rows: expand: s = z / T, [row][V]; zdump: z, [aux][V];
-  // qrows: q = exp(s - lse), [b][Nmax+1][V] with row aux
+  // expand: one partial per (node row, CTA), index row * ncta_v + cta
+  float2* pstats;        // (max, sum exp(s - max)) of the CTA's vocabulary range
+  float* plv;            // [k] top-k values of s, best first (ties: lower token)
+  int32_t* pli;          // [k] their tokens
+  float* pgv;            // [k] Gumbel-top-k keys (T > 0)
+  int32_t* pgi;          // [k] their tokens
+  // zdump: z, [aux][ldo] (fp32, or bf16 if out_bf16); qrows: q = exp(s - lse),
+  // [b][Nmax+1][ldo] with row aux; swiglu: silu(gate) * up, bf16 [aux][ldo]
   float* out;
+  int ldo;               // output row stride in elements (0: V)
+  int out_bf16;
   int nmax1;             // Nmax + 1
   int32_t* status;
   int stages;
-};
-
-struct TopkArgs {
-  const float* S;        // [Mcap][V] scaled logits of this wave's nodes
-  const Row* rows;
-  const int32_t* n_rows;
-  int Mcap, V, k, nchunk, chunk;
-  float temp;
-  uint64_t seed;
-  uint32_t offset;
-  float2* stats;         // [Mcap][nchunk] (max, sum exp(s - max))
-  float* lv;             // [Mcap][nchunk][k] top-k of s
-  int32_t* li;
-  float* gv;             // [Mcap][nchunk][k] Gumbel top-k (T > 0)
-  int32_t* gi;
-  int32_t* row_done;     // [Mcap] chunks finished per row (the last one merges and resets)
-  float* fin_lse;        // [Mcap] merged results per node
-  float* fin_v;          // [Mcap][k] top-k values of s (order statistics)
-  int32_t* fin_i;        // [Mcap][k] their tokens
-  int32_t* fin_g;        // [Mcap][k] Gumbel-top-k tokens (T > 0)
-  int32_t* status;
 };
 
 struct FrontierArgs {
@@ -102,10 +91,12 @@ struct FrontierArgs {
   const uint16_t* A;     // [V][r]
   ReqState* req;
   Cand* lists;           // [batch][Nmax]
-  const float* fin_lse;  // [Mcap] per expanded node: log-sum-exp of s
-  const float* fin_v;    // [Mcap][k] top-k values of s
-  const int32_t* fin_i;  // [Mcap][k] their tokens
-  const int32_t* fin_g;  // [Mcap][k] Gumbel-top-k tokens (T > 0)
+  const float2* pstats;  // per-CTA partials of the wave GEMM (see GemmArgs)
+  const float* plv;
+  const int32_t* pli;
+  const float* pgv;
+  const int32_t* pgi;
+  int ncta;              // partials per node
   const float* calib;    // [Bk][2] or NULL
   const int32_t* n_budget;
   const int32_t* k_req;

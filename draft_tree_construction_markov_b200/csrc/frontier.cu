@@ -13,6 +13,7 @@
 // kept set is the sequential result; and a node outside the top-N of a subset
 // of candidates is outside the top-N of any superset, so at most Bk waves run.
 #include "build.cuh"
+#include "merge.cuh"
 
 namespace dt {
 
@@ -32,6 +33,7 @@ __device__ __forceinline__ void gather_row(uint16_t* dst, const uint16_t* A, int
   for (int i = lane; i < r / 8; i += nlanes) d[i] = s[i];
 }
 
+template <int KMAX>
 __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs f) {
   extern __shared__ __align__(16) uint8_t fsm[];
   const int b = blockIdx.x;
@@ -62,18 +64,26 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
   for (int i = tid; i < n_old; i += kFrontierThreads) cands[i] = f.lists[(size_t)b * Nmax + i];
   for (int i = tid; i < rows_n; i += kFrontierThreads) s_rows[i] = f.rows[st.row_base + i];
   if (tid < 4) s_cnt[tid] = 0;
-  // the merged per-node results come from the top-k pass launched just before
+  // the per-CTA partials come from the wave GEMM launched just before
   pdl_wait();
   pdl_launch_dependents();
 
-  // 1. each expanded node's log-sum-exp and its k best (or sampled) children
-  for (int i = tid; i < rows_n * kb; i += kFrontierThreads) {
-    const int e = i / kb, j = i % kb;
-    const int row = st.row_base + e;
-    const float lse = f.fin_lse[row];
-    if (j == 0) r_lse[e] = lse;
-    r_lq[e * k + j] = f.fin_v[(size_t)row * k + j] - lse;
-    r_tok[e * k + j] = f.temp > 0.f ? f.fin_g[(size_t)row * k + j] : f.fin_i[(size_t)row * k + j];
+  // 1. merge each expanded node's partials: its log-sum-exp and its kb best
+  // (T = 0) or sampled (T > 0, Gumbel-top-k) children, one warp per node
+  for (int e = warp; e < rows_n; e += kWarps) {
+    const size_t prow = (size_t)(st.row_base + e) * f.ncta;
+    const float lse = merge_lse(f.pstats + prow, f.ncta, lane);
+    // values of the k best (order statistics of s); tokens of the best (T = 0)
+    // or of the Gumbel sample (T > 0)
+    const bool stoch = f.temp > 0.f;
+    merge_lists<KMAX>(f.plv + prow * k, f.pli + prow * k, f.ncta, k, kb, lane, r_lq + e * k,
+                      stoch ? nullptr : r_tok + e * k);
+    if (stoch)
+      merge_lists<KMAX>(f.pgv + prow * k, f.pgi + prow * k, f.ncta, k, kb, lane, nullptr,
+                        r_tok + e * k);
+    __syncwarp();
+    if (lane == 0) r_lse[e] = lse;
+    for (int j = lane; j < kb; j += 32) r_lq[e * k + j] -= lse;
   }
   __syncthreads();
 
@@ -349,11 +359,14 @@ size_t frontier_smem_bytes(int Nmax, int k) {
          (size_t)Nmax * 4 + (size_t)Nmax * k * 4 * 2;
 }
 
+int gemm_kmax(int k);
+
 cudaError_t launch_frontier(const FrontierArgs& f, cudaStream_t s) {
   const size_t smem = frontier_smem_bytes(f.Nmax, f.k);
-  cudaError_t e = ensure_smem(frontier_kernel, smem);
+  auto kern = gemm_kmax(f.k) == 4 ? frontier_kernel<4> : frontier_kernel<16>;
+  cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(frontier_kernel, dim3(f.batch), dim3(kFrontierThreads), smem, s, f);
+  e = launch_pdl(kern, dim3(f.batch), dim3(kFrontierThreads), smem, s, f);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

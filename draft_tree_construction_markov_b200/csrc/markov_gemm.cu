@@ -1,43 +1,74 @@
-// Parent-conditioned logits on the 5th-generation tensor cores.
+// Node-batched GEMMs on the 5th-generation tensor cores, with fused epilogues.
 //
-// For every GEMM column n (a tree node u with depth d and token t) and every
-// vocabulary row x:
+// Markov head (PCTree summary, DSpark paragraph: the Markov head biases the
+// shared block logits by the previous token; here the previous token is the
+// node's own token, i.e. the children are parent-conditioned).  For every
+// GEMM column n (a tree node u with depth d and token t) and every vocabulary
+// row x:
 //   z[x][n] = L[b][d][x] + sum_rho Bm[x][rho] * A[t][rho]
-// (PCTree summary, DSpark paragraph: the Markov head biases the shared block
-// logits by the previous token; here the previous token is the node's own
-// token, i.e. the children are parent-conditioned.)
+// The same kernel serves the TreeFlash AR-approximator (TreeFlash explainer,
+// method section 1): the SwiGLU gate/up projections, the down projection
+// with the residual, and the LM head, whose columns are approximator rows.
 //
-// Swap-AB tcgen05 GEMM: the vocabulary is the MMA M axis (128 rows per tile,
-// the Markov factor Bm streamed by TMA), nodes are the N axis (the gathered
-// rows A[t], also by TMA), K = r.  The fp32 accumulator lives in TMEM (double
-// buffered); epilogue warps read it back with tcgen05.ld, one 32-lane quadrant
-// each (lane = vocabulary row), add the block-logit bias and store one fp32
-// row per node: s = z / T for the top-k pass (EXPAND), z itself (ZDUMP) or
-// q = exp(s - lse) (QROWS).  Columns without a node are skipped.  Each CTA
-// owns a contiguous range of vocabulary tiles.
+// Swap-AB tcgen05 GEMM: the weight rows (vocabulary, or features) are the MMA
+// M axis (128 rows per tile, streamed by TMA), node rows are the N axis (32,
+// 64 or 256 per tile, also by TMA), K is the inner dimension.  The fp32
+// accumulator lives in TMEM, two or four tiles deep, so the tensor pipe runs
+// ahead of the epilogue.  Each CTA owns a contiguous range of weight tiles and
+// one node tile; CTAs of the same range are adjacent in the grid, so the
+// weight tiles that several node tiles share are re-read from L2.
+//
+// Epilogues:
+//  * EXPAND (the hot path of both trees): four warps per 32 node columns read
+//    the accumulator back with tcgen05.ld (each warp its 32-lane quadrant = 32
+//    vocabulary rows) and transpose each 32 x 32 block through shared memory,
+//    so every thread owns ONE node column and scans 32 consecutive vocabulary
+//    entries of it per tile.  Per column it fuses the block-logit bias
+//    (prefetched one tile ahead), the temperature, a batched max / sum-exp, a
+//    private top-k of s (ties to the lower token id) and, at T > 0, the
+//    Gumbel-top-k of s + G (TreeSpark article, "lossless" section;
+//    Gumbel-top-k: Kool, van Hoof and Welling 2019), one Philox call per four
+//    consecutive tokens.  The CTA writes one partial result per node; a later
+//    kernel merges the partials.
+//  * ZDUMP: z (+ optional bias rows), fp32 or bf16, lane = weight row so that
+//    stores coalesce.  Also the down projection + residual of TreeFlash.
+//  * QROWS: q = exp(s - lse) rows of the final tree (T > 0).
+//  * SWIGLU: a tile holds 64 gate rows (TMEM lanes 0-63) and the 64 up rows of
+//    the same features (lanes 64-127); the up quadrants hand their values to
+//    the gate quadrants through shared memory, which store silu(g) * u (bf16).
 #include "build.cuh"
 
 namespace dt {
 
 constexpr int kTileV = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+// U <= 1 - 2^-24 gives G = -log(-log U) <= 16.64; tokens with s + 16.75 below
+// the current k-th Gumbel key cannot enter the sample and skip the Philox draw.
+constexpr float kGumbelMax = 16.75f;
+constexpr int kTLD = 33;  // transpose buffer row stride (floats)
 
-// NG groups of 32 node columns per tile; every epilogue warp reads CW columns
-// of one 32-lane TMEM quadrant, so each quadrant is served by NT / CW warps.
-template <int NG, int CW>
+// NG groups of 32 node columns per tile.  The epilogue serves EG groups at a
+// time with four warps each (one per TMEM lane quadrant); each epilogue thread
+// handles CPT groups of its quadrant in turn.
+template <int NG>
 struct GemmShape {
   static constexpr int NT = 32 * NG;  // MMA N: node columns per tile
-  static constexpr int EPQ = NT / CW;  // epilogue warps per quadrant
-  static constexpr int kEpiWarps = 4 * EPQ;
+  static constexpr int EG = NG < 2 ? NG : 2;
+  static constexpr int CPT = NG / EG;
+  static constexpr int kEpiWarps = 4 * EG;
   static constexpr int kThreads = 32 * (2 + kEpiWarps);
-  static constexpr int kABytes = kTileV * 128;  // 128 vocab rows x 64 bf16
-  static constexpr int kBBytes = NT * 128;      // NT node rows x 64 bf16
+  static constexpr int kAccBufs = NG <= 2 ? 4 : 2;  // accumulator tiles in TMEM
+  static constexpr int kABytes = kTileV * 128;      // 128 weight rows x 64 bf16
+  static constexpr int kBBytes = NT * 128;          // NT node rows x 64 bf16
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kTmemCols = (2 * NT <= 64) ? 64 : (2 * NT <= 128) ? 128 : 256;
-  static_assert(NT % 16 == 0 && NT <= 256, "MMA N must be a multiple of 16, at most 256");
+  static constexpr uint32_t kTmemCols = kAccBufs * NT;
+  static_assert(NG == 1 || NG == 2 || NG == 8, "node tile of 32, 64 or 256 columns");
+  static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512,
+                "TMEM allocation is a power of two");
 };
 
 struct ColMeta {
-  int64_t bias_off;  // element offset of the node's block-logit row
+  int64_t bias_off;  // element offset of the column's bias row (block logits / residual)
   uint32_t c1, c2;   // Philox counter words 1-2 (path id)
   int32_t b;
   int32_t valid;
@@ -45,32 +76,138 @@ struct ColMeta {
   int32_t out_row;
 };
 
-template <int NG, int CW>
-static size_t gemm_smem_bytes(int stages) {
-  using S = GemmShape<NG, CW>;
+template <int NG>
+static size_t gemm_epi_bytes(int mode, int kmax, bool stoch) {
+  using S = GemmShape<NG>;
+  const size_t tbuf = (size_t)S::kEpiWarps * 32 * kTLD * 4;
+  if (mode == EPI_SWIGLU) return tbuf;
+  if (mode != EPI_EXPAND) return 0;
+  // after the tile loop the transpose buffers hold the per-quadrant partials
+  const size_t lists = (size_t)4 * S::NT * kmax * 8 * (stoch ? 2 : 1) + (size_t)4 * S::NT * 8;
+  return tbuf > lists ? tbuf : lists;
+}
+
+template <int NG>
+static size_t gemm_smem_bytes(int stages, int mode, int kmax, bool stoch) {
+  using S = GemmShape<NG>;
   size_t off = 1024;  // alignment slack
   off += (size_t)stages * S::kStageBytes;
-  off += (size_t)(2 * stages + 5) * 8;  // barriers
-  off += 16;                             // tmem slot + abort flag
+  off += (size_t)(2 * stages + 2 * S::kAccBufs + 5) * 8;  // barriers
+  off += 16;                                             // tmem slot + abort flag
   off = (off + 15) & ~(size_t)15;
   off += (size_t)S::NT * sizeof(ColMeta);
+  off += gemm_epi_bytes<NG>(mode, kmax, stoch);
   return off;
 }
 
-template <int NG, int CW, int MODE, bool STOCH>
-__global__ void __launch_bounds__(GemmShape<NG, CW>::kThreads, 1)
+// Insert (v, id) into a register list sorted by value (descending) when ids
+// arrive in increasing order: equal values keep their earlier entries first.
+// Entries past k are scratch.  Caller guarantees v > list[k-1].
+template <int KMAX>
+__device__ __forceinline__ void topk_insert(float (&L)[KMAX], int32_t (&I)[KMAX], float v,
+                                            int32_t id) {
+  float nl[KMAX];
+  int32_t ni[KMAX];
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    const bool ge = L[i] >= v;
+    const bool gep = (i == 0) ? false : (L[i - 1] >= v);
+    nl[i] = ge ? L[i] : ((i == 0 || gep) ? v : L[i - 1]);
+    ni[i] = ge ? I[i] : ((i == 0 || gep) ? id : I[i - 1]);
+  }
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    L[i] = nl[i];
+    I[i] = ni[i];
+  }
+}
+
+template <int KMAX>
+__device__ __forceinline__ float kth(const float (&L)[KMAX], int k) {
+  float t = L[0];
+#pragma unroll
+  for (int i = 1; i < KMAX; ++i)
+    if (i == k - 1) t = L[i];
+  return t;
+}
+
+// (v1, i1) ranks before (v2, i2): larger value first, then lower id.
+__device__ __forceinline__ bool ranks_before(float v1, int32_t i1, float v2, int32_t i2) {
+  return v1 > v2 || (v1 == v2 && i1 < i2);
+}
+
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Raw 128 bytes of a bias row (32 fp32 or the first 64 bytes = 32 bf16).
+__device__ __forceinline__ void load_bias_raw(const void* L, int bf16, int64_t off,
+                                              uint4 (&raw)[8]) {
+  const uint4* p =
+      bf16 ? (const uint4*)((const uint16_t*)L + off) : (const uint4*)((const float*)L + off);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    if (c < 4 || !bf16) raw[c] = __ldg(p + c);
+}
+
+__device__ __forceinline__ void decode_bias(const uint4 (&raw)[8], int bf16, float (&bias)[32]) {
+  if (bf16) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        bias[8 * c + 2 * h] = __uint_as_float(w[h] << 16);
+        bias[8 * c + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      bias[4 * c] = __uint_as_float(raw[c].x);
+      bias[4 * c + 1] = __uint_as_float(raw[c].y);
+      bias[4 * c + 2] = __uint_as_float(raw[c].z);
+      bias[4 * c + 3] = __uint_as_float(raw[c].w);
+    }
+  }
+}
+
+__device__ __forceinline__ float load_bias1(const void* L, int bf16, int64_t off) {
+  return bf16 ? bf16_to_f32(__ldg((const uint16_t*)L + off)) : __ldg((const float*)L + off);
+}
+
+// fp32 -> bf16, round to nearest even (finite inputs).
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (uint16_t)((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+}
+
+// 32 lanes x 32 columns of 32-bit TMEM cells -> 32 registers per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&acc)[32]) {
+  float v[16];
+  tmem_ld16(taddr, v);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = v[i];
+  tmem_ld16(taddr + 16, v);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[16 + i] = v[i];
+}
+
+template <int NG, int MODE, bool STOCH, int KMAX>
+__global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
     markov_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
+                       const __grid_constant__ CUtensorMap tmW2,
                        const __grid_constant__ CUtensorMap tmH, GemmArgs a, int batch) {
-  using S = GemmShape<NG, CW>;
+  using S = GemmShape<NG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cx = blockIdx.x, ny = blockIdx.y;
-  // the node rows, their count and the gathered Markov rows come from the
-  // previous kernel
+  // node tile fastest: the CTAs that share a weight range run side by side
+  const int cx = blockIdx.x / a.n_ntiles, ny = blockIdx.x % a.n_ntiles;
+  // the node rows, their count and the gathered rows come from the previous kernel
   pdl_wait();
   const int M = min(*a.n_rows, a.Mcap);
-  if (cx == 0 && ny == 0 && threadIdx.x == 0 && a.reset_count) *a.reset_count = 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && a.reset_count) *a.reset_count = 0;
   pdl_launch_dependents();
   if (ny * S::NT >= M) return;  // uniform over the CTA
 
@@ -80,6 +217,7 @@ __global__ void __launch_bounds__(GemmShape<NG, CW>::kThreads, 1)
   const int KC = (a.r + 63) >> 6;
   const int ks_last = (((a.r - 1) & 63) >> 4) + 1;
   const int stages = a.stages;
+  const int k = a.k;
 
   // ---- carve shared memory
   uint8_t* p = smem;
@@ -88,30 +226,39 @@ __global__ void __launch_bounds__(GemmShape<NG, CW>::kThreads, 1)
   uint64_t* full = (uint64_t*)p;
   uint64_t* empty = full + stages;
   uint64_t* tfull = empty + stages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  p = (uint8_t*)(drain + 1);
+  uint64_t* tempty = tfull + S::kAccBufs;
+  uint64_t* drain = tempty + S::kAccBufs;
+  uint64_t* xfull = drain + 1;   // [2] SwiGLU: up values staged for column group eg
+  uint64_t* xempty = xfull + 2;  // [2] SwiGLU: staged values consumed
+  p = (uint8_t*)(xempty + 2);
   uint32_t* tmem_slot = (uint32_t*)p;
   volatile int* abort_flag = (volatile int*)(p + 4);
   p += 16;
   p = (uint8_t*)(((uintptr_t)p + 15) & ~(uintptr_t)15);
   ColMeta* meta = (ColMeta*)p;
   p += S::NT * sizeof(ColMeta);
+  float* tbuf = (float*)p;  // [kEpiWarps][32][kTLD]; EXPAND: then the quadrant partials
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < S::kAccBufs; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], S::kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&xfull[i], 64);
+      mbar_init(&xempty[i], 64);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmW);
+    if (MODE == EPI_SWIGLU) prefetch_tmap(&tmW2);
     prefetch_tmap(&tmH);
   }
   for (int c = threadIdx.x; c < S::NT; c += blockDim.x) {
@@ -164,7 +311,13 @@ __global__ void __launch_bounds__(GemmShape<NG, CW>::kThreads, 1)
           }
           uint8_t* sa = stage_mem + (size_t)stage * S::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
-          tma_load_2d(sa, &tmW, &full[stage], kc * 64, t * kTileV);
+          if (MODE == EPI_SWIGLU) {
+            // 64 gate rows, then the 64 up rows of the same features
+            tma_load_2d(sa, &tmW, &full[stage], kc * 64, t * 64);
+            tma_load_2d(sa + S::kABytes / 2, &tmW2, &full[stage], kc * 64, t * 64);
+          } else {
+            tma_load_2d(sa, &tmW, &full[stage], kc * 64, t * kTileV);
+          }
           tma_load_2d(sa + S::kABytes, &tmH, &full[stage], kc * 64, ny * S::NT);
           issued |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -218,8 +371,10 @@ __global__ void __launch_bounds__(GemmShape<NG, CW>::kThreads, 1)
         }
         if (!ok) break;
         tc_commit(&tfull[ab]);
-        ab ^= 1;
-        if (ab == 0) aphase ^= 1;
+        if (++ab == S::kAccBufs) {
+          ab = 0;
+          aphase ^= 1;
+        }
       }
       // every MMA issued by this thread has completed once `drain` flips
       tc_commit(drain);
@@ -227,63 +382,316 @@ __global__ void __launch_bounds__(GemmShape<NG, CW>::kThreads, 1)
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t_start < kWaitLimitNs) {
       }
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    // Warp e reads TMEM quadrant q (vocabulary rows 32q..32q+31 of each tile;
-    // lane = row) for the CW node columns of group cg; stores coalesce.
+  } else if (MODE == EPI_ZDUMP || MODE == EPI_QROWS) {
+    // ------------------------------------- z / draft-q epilogue (lane = row)
     const int e = warp - 2;
-    const int q = warp & 3;
-    const int cg = e >> 2;
-    const float temp = a.temp;
+    const int q = warp & 3;  // TMEM lane quadrant accessible to this warp
+    const int eg = e >> 2;   // column group served by this warp
     int ab = 0;
     uint32_t aphase = 0;
     for (int t = t0; t < t1; ++t) {
-      const int x0 = t * kTileV + 32 * q;
-      const int x = x0 + lane;
-      const bool xin = x < a.V;
-      // block-logit bias of every node column of this tile, loaded before
-      // waiting for the accumulator so the latency overlaps the MMA
-      float bias[CW];
-#pragma unroll
-      for (int j = 0; j < CW; ++j) {
-        const ColMeta& cm = meta[cg * CW + j];
-        bias[j] = 0.f;
-        if (cm.valid && xin)
-          bias[j] = a.l_bf16 ? bf16_to_f32(__ldg((const uint16_t*)a.L + cm.bias_off + x))
-                             : __ldg((const float*)a.L + cm.bias_off + x);
-      }
+      const int x = t * kTileV + 32 * q + lane;
       if (!mbar_wait(&tfull[ab], aphase, a.status, abort_flag)) break;
       tc_fence_after();
-      float acc[CW];
-      const uint32_t taddr =
-          tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * S::NT + cg * CW);
+#pragma unroll 1
+      for (int j = 0; j < S::CPT; ++j) {
+        const int grp = eg + j * S::EG;
+        float acc[32];
+        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * S::NT + grp * 32), acc);
+        if (j == S::CPT - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[ab]);
+        }
+        if (x >= a.V) continue;
 #pragma unroll
-      for (int c = 0; c < CW / 16; ++c) {
-        float v[16];
-        tmem_ld16(taddr + 16 * c, v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) acc[16 * c + i] = v[i];
+        for (int i = 0; i < 32; ++i) {
+          const ColMeta& cm = meta[grp * 32 + i];
+          if (!cm.valid) continue;  // warp-uniform
+          const float bias = a.L ? load_bias1(a.L, a.l_bf16, cm.bias_off + x) : 0.f;
+          const float z = acc[i] + bias;
+          if (MODE == EPI_ZDUMP) {
+            if (a.out_bf16)
+              ((uint16_t*)a.out)[(size_t)cm.out_row * a.ldo + x] = f32_to_bf16_rne(z);
+            else
+              a.out[(size_t)cm.out_row * a.ldo + x] = z;
+          } else {
+            a.out[((size_t)cm.b * a.nmax1 + cm.out_row) * a.ldo + x] =
+                expf(__fdiv_rn(z, a.temp) - cm.lse);
+          }
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[ab]);
-      ab ^= 1;
-      if (ab == 0) aphase ^= 1;
-      if (!xin) continue;
+      if (++ab == S::kAccBufs) {
+        ab = 0;
+        aphase ^= 1;
+      }
+    }
+  } else if (MODE == EPI_SWIGLU) {
+    // -------------------------- SwiGLU epilogue: silu(gate) * up, bf16 rows
+    // The two up warps of column group eg stage their values in their own
+    // transpose buffers (xfull), the two gate warps consume them (xempty);
+    // every wait is bounded, so a timed-out warp cannot strand the others.
+    const int e = warp - 2;
+    const int q = warp & 3;
+    const int eg = e >> 2;
+    const bool up = q >= 2;  // TMEM lanes 64-127 hold the up projection
+    // warp e = 4 eg + ((q - 2) & 3); the up warp of quadrant q + 2 is 4 eg + q
+    float* tb_own = tbuf + (size_t)e * 32 * kTLD;
+    float* tb_up = tbuf + (size_t)(4 * eg + (q & 1)) * 32 * kTLD;
+    int ab = 0;
+    uint32_t aphase = 0;
+    uint32_t xn = 0;  // exchanges so far (phase parity)
+    bool ok = true;
+    for (int t = t0; t < t1 && ok; ++t) {
+      const int f = t * 64 + 32 * (q & 1) + lane;  // feature of this lane
+      if (!mbar_wait(&tfull[ab], aphase, a.status, abort_flag)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int j = 0; j < S::CPT; ++j, ++xn) {
+        const int grp = eg + j * S::EG;
+        float acc[32];
+        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * S::NT + grp * 32), acc);
+        if (j == S::CPT - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[ab]);
+        }
+        if (up) {
+          if (!mbar_wait(&xempty[eg], (xn & 1) ^ 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
 #pragma unroll
-      for (int j = 0; j < CW; ++j) {
-        const int c = cg * CW + j;
-        const ColMeta& cm = meta[c];
-        if (!cm.valid) continue;  // warp-uniform
-        const float z = acc[j] + bias[j];
-        if (MODE == EPI_ZDUMP) {
-          a.out[(size_t)cm.out_row * a.V + x] = z;
+          for (int i = 0; i < 32; ++i) tb_own[lane * kTLD + i] = acc[i];
+          mbar_arrive(&xfull[eg]);
         } else {
-          const float s = STOCH ? __fdiv_rn(z, temp) : z;
-          if (MODE == EPI_QROWS)
-            a.out[((size_t)cm.b * a.nmax1 + cm.out_row) * a.V + x] = expf(s - cm.lse);
-          else  // EPI_EXPAND: the scaled logits, one fp32 row per GEMM column
-            a.out[(size_t)(ny * S::NT + c) * a.V + x] = s;
+          if (!mbar_wait(&xfull[eg], xn & 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (f < a.V) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const ColMeta& cm = meta[grp * 32 + i];
+              if (!cm.valid) continue;  // warp-uniform
+              const float g = acc[i];
+              const float u = tb_up[lane * kTLD + i];
+              const float act = __fdiv_rn(g, 1.f + expf(-g)) * u;
+              ((uint16_t*)a.out)[(size_t)cm.out_row * a.ldo + f] = f32_to_bf16_rne(act);
+            }
+          }
+          mbar_arrive(&xempty[eg]);
+        }
+      }
+      if (++ab == S::kAccBufs) {
+        ab = 0;
+        aphase ^= 1;
+      }
+    }
+  } else {
+    // --------------------------------------------- expansion epilogue (columns)
+    const int e = warp - 2;
+    const int q = warp & 3;  // TMEM lane quadrant accessible to this warp
+    const int eg = e >> 2;   // first column group of this warp
+    const float temp = a.temp;
+    float* tb = tbuf + (size_t)e * 32 * kTLD;
+    ColMeta mc[S::CPT];
+#pragma unroll
+    for (int j = 0; j < S::CPT; ++j) mc[j] = meta[(eg + j * S::EG) * 32 + lane];
+    float m[S::CPT], ssum[S::CPT], thr[S::CPT], gthr[S::CPT];
+    float L1[S::CPT][KMAX];
+    int32_t I1[S::CPT][KMAX];
+    float L2[S::CPT][KMAX];
+    int32_t I2[S::CPT][KMAX];
+#pragma unroll
+    for (int j = 0; j < S::CPT; ++j) {
+      m[j] = -INFINITY;
+      ssum[j] = 0.f;
+      thr[j] = -INFINITY;
+      gthr[j] = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < KMAX; ++i) {
+        L1[j][i] = -INFINITY;
+        I1[j][i] = 0x7fffffff;
+        L2[j][i] = -INFINITY;
+        I2[j][i] = 0x7fffffff;
+      }
+    }
+    // bias rows (one column group per thread only): requested one tile ahead
+    const bool has_bias = S::CPT == 1 && a.L != nullptr;
+    const bool vec = a.l_vec != 0;
+    uint4 raw[8];
+    bool raw_ok = false;
+    if (has_bias) {
+      const int xq = t0 * kTileV + 32 * q;
+      raw_ok = mc[0].valid && vec && xq + 32 <= a.V && t0 < t1;
+      if (raw_ok) load_bias_raw(a.L, a.l_bf16, mc[0].bias_off + xq, raw);
+    }
+    int ab = 0;
+    uint32_t aphase = 0;
+    for (int t = t0; t < t1; ++t) {
+      if (!mbar_wait(&tfull[ab], aphase, a.status, abort_flag)) break;
+      tc_fence_after();
+      const int xq = t * kTileV + 32 * q;  // first vocabulary row of this quadrant
+      const int nv = min(32, a.V - xq);
+#pragma unroll
+      for (int j = 0; j < S::CPT; ++j) {
+        const int grp = eg + j * S::EG;
+        float acc[32];
+        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * S::NT + grp * 32), acc);
+        if (j == S::CPT - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[ab]);
+        }
+        float bias[32];
+        bool had_raw = false;
+        if (has_bias) {
+          if (raw_ok) decode_bias(raw, a.l_bf16, bias);
+          had_raw = raw_ok;
+          const int xn = xq + kTileV;
+          raw_ok = mc[0].valid && vec && t + 1 < t1 && xn + 32 <= a.V;
+          if (raw_ok) load_bias_raw(a.L, a.l_bf16, mc[0].bias_off + xn, raw);
+        }
+        // transpose 32 rows x 32 columns: thread `lane` takes column grp*32+lane
+#pragma unroll
+        for (int i = 0; i < 32; ++i) tb[lane * kTLD + i] = acc[i];
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = tb[i * kTLD + lane];
+        __syncwarp();
+        if (!mc[j].valid || nv <= 0) continue;
+        if (!has_bias) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) bias[i] = 0.f;
+        } else if (!had_raw) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            bias[i] = i < nv ? load_bias1(a.L, a.l_bf16, mc[j].bias_off + xq + i) : 0.f;
+        }
+        float s[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float z = acc[i] + bias[i];
+          s[i] = i < nv ? (STOCH ? __fdiv_rn(z, temp) : z) : -INFINITY;
+        }
+        // log-sum-exp, batched over the 32 values
+        float mt = s[0];
+#pragma unroll
+        for (int i = 1; i < 32; ++i) mt = fmaxf(mt, s[i]);
+        float st = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) st += exp2f((s[i] - mt) * kLog2e);
+        if (mt > m[j]) {
+          ssum[j] = ssum[j] * exp2f((m[j] - mt) * kLog2e) + st;
+          m[j] = mt;
+        } else {
+          ssum[j] += st * exp2f((mt - m[j]) * kLog2e);
+        }
+        // top-k of s (values arrive in increasing token order)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (s[i] > thr[j]) {
+            topk_insert<KMAX>(L1[j], I1[j], s[i], xq + i);
+            thr[j] = kth<KMAX>(L1[j], k);
+          }
+        }
+        if constexpr (STOCH) {
+          // Gumbel keys; four consecutive tokens share one Philox counter
+#pragma unroll
+          for (int gi = 0; gi < 8; ++gi) {
+            const float smax =
+                fmaxf(fmaxf(s[4 * gi], s[4 * gi + 1]), fmaxf(s[4 * gi + 2], s[4 * gi + 3]));
+            if (!(smax + kGumbelMax > gthr[j])) continue;
+            const uint32_t x4 = (uint32_t)(xq + 4 * gi);
+            const U4 o =
+                philox10(U4{(x4 >> 2) | ((uint32_t)mc[j].b << 18), mc[j].c1, mc[j].c2, a.offset},
+                         (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
+            const uint32_t wds[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const int i = 4 * gi + jj;
+              if (i >= nv) continue;
+              const float gk = s[i] + (-logf(-logf(u23(wds[jj]))));
+              if (gk > gthr[j]) {
+                topk_insert<KMAX>(L2[j], I2[j], gk, xq + i);
+                gthr[j] = kth<KMAX>(L2[j], k);
+              }
+            }
+          }
+        }
+      }
+      if (++ab == S::kAccBufs) {
+        ab = 0;
+        aphase ^= 1;
+      }
+    }
+    // publish this quadrant's partials of the owned columns (the transpose
+    // buffers are free once every epilogue warp has left the tile loop)
+    named_bar(1, S::kEpiWarps * 32);
+    float* ql1v = tbuf;  // [4][NT][KMAX] per-quadrant top-k of s
+    int32_t* ql1i = (int32_t*)(ql1v + 4 * S::NT * KMAX);
+    float* ql2v = (float*)(ql1i + 4 * S::NT * KMAX);  // Gumbel lists (T > 0)
+    int32_t* ql2i = (int32_t*)(ql2v + (STOCH ? 4 * S::NT * KMAX : 0));
+    float2* qst = (float2*)(ql2i + (STOCH ? 4 * S::NT * KMAX : 0));  // [4][NT]
+#pragma unroll
+    for (int j = 0; j < S::CPT; ++j) {
+      const int col = (eg + j * S::EG) * 32 + lane;
+      qst[q * S::NT + col] = make_float2(m[j], ssum[j]);
+#pragma unroll
+      for (int i = 0; i < KMAX; ++i) {
+        ql1v[(q * S::NT + col) * KMAX + i] = L1[j][i];
+        ql1i[(q * S::NT + col) * KMAX + i] = I1[j][i];
+        if (STOCH) {
+          ql2v[(q * S::NT + col) * KMAX + i] = L2[j][i];
+          ql2i[(q * S::NT + col) * KMAX + i] = I2[j][i];
+        }
+      }
+    }
+    named_bar(1, S::kEpiWarps * 32);
+    // one thread per column merges the four quadrants into the CTA's partial
+    const int et = threadIdx.x - 64;
+    for (int c = et; c < S::NT; c += S::kEpiWarps * 32) {
+      if (!meta[c].valid) continue;
+      const int row = ny * S::NT + c;
+      float mx = -INFINITY;
+      for (int qq = 0; qq < 4; ++qq) mx = fmaxf(mx, qst[qq * S::NT + c].x);
+      float sv = 0.f;
+      if (mx != -INFINITY)
+        for (int qq = 0; qq < 4; ++qq) {
+          const float2 rv = qst[qq * S::NT + c];
+          if (rv.x != -INFINITY) sv += rv.y * exp2f((rv.x - mx) * kLog2e);
+        }
+      const size_t pidx = (size_t)row * a.ncta_v + cx;
+      a.pstats[pidx] = make_float2(mx, sv);
+      for (int lst = 0; lst < (STOCH ? 2 : 1); ++lst) {
+        const float* LV = lst ? ql2v : ql1v;
+        const int32_t* LI = lst ? ql2i : ql1i;
+        float* OV = (lst ? a.pgv : a.plv) + pidx * k;
+        int32_t* OI = (lst ? a.pgi : a.pli) + pidx * k;
+        int h0 = 0, h1 = 0, h2 = 0, h3 = 0;  // heads of the four quadrant lists
+        for (int i = 0; i < k; ++i) {
+          int bw = -1;
+          float bv = -INFINITY;
+          int32_t bi = 0x7fffffff;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int hw = w == 0 ? h0 : w == 1 ? h1 : w == 2 ? h2 : h3;
+            if (hw >= k) continue;
+            const float v = LV[(w * S::NT + c) * KMAX + hw];
+            const int32_t id = LI[(w * S::NT + c) * KMAX + hw];
+            if (bw < 0 || ranks_before(v, id, bv, bi)) {
+              bw = w;
+              bv = v;
+              bi = id;
+            }
+          }
+          h0 += bw == 0;
+          h1 += bw == 1;
+          h2 += bw == 2;
+          h3 += bw == 3;
+          OV[i] = bv;
+          OI[i] = bi;
         }
       }
     }
@@ -329,43 +737,61 @@ bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t K, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NG, int CW, int MODE, bool STOCH>
-static cudaError_t launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmH, GemmArgs a,
-                              int batch, int n_node_tiles, cudaStream_t s) {
-  using SH = GemmShape<NG, CW>;
-  auto kern = markov_gemm_kernel<NG, CW, MODE, STOCH>;
+template <int NG, int MODE, bool STOCH, int KMAX>
+static cudaError_t launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmW2,
+                              const CUtensorMap& tmH, GemmArgs a, int batch, cudaStream_t s) {
+  using SH = GemmShape<NG>;
+  auto kern = markov_gemm_kernel<NG, MODE, STOCH, KMAX>;
   // the deepest pipeline that fits in 220 KB of shared memory
-  int stages = 8;
-  while (stages > 2 && gemm_smem_bytes<NG, CW>(stages) > 220 * 1024) --stages;
+  int stages = 10;
+  while (stages > 2 && gemm_smem_bytes<NG>(stages, MODE, KMAX, STOCH) > 220 * 1024) --stages;
   a.stages = stages;
-  const size_t smem = gemm_smem_bytes<NG, CW>(stages);
+  const size_t smem = gemm_smem_bytes<NG>(stages, MODE, KMAX, STOCH);
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.ncta_v, n_node_tiles);
-  e = launch_pdl(kern, grid, dim3(SH::kThreads), smem, s, tmW, tmH, a, batch);
+  const dim3 grid(a.ncta_v * a.n_ntiles);
+  e = launch_pdl(kern, grid, dim3(SH::kThreads), smem, s, tmW, tmW2, tmH, a, batch);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 // Node columns per tile the launcher uses for a given column capacity.
-int gemm_node_tile(int max_cols) { return max_cols <= 32 ? 32 : 64; }
+int gemm_node_tile(int max_cols) { return max_cols <= 32 ? 32 : max_cols <= 64 ? 64 : 256; }
 
+// Largest top-k list a launch keeps per column for k children per node.
+int gemm_kmax(int k) { return k <= 4 ? 4 : 16; }
+
+// Launches one GEMM.  tmW: weight rows (box 128 rows; SwiGLU: the gate rows,
+// box 64, with tmW2 the up rows); tmH: node rows (box nt rows).
 cudaError_t launch_markov_gemm(int mode, bool stoch, const CUtensorMap& tmW,
-                               const CUtensorMap& tmH, const GemmArgs& a, int batch, int nt,
-                               cudaStream_t s) {
-  const int ntiles = (a.Mcap + nt - 1) / nt;
+                               const CUtensorMap& tmW2, const CUtensorMap& tmH, GemmArgs a,
+                               int batch, int nt, cudaStream_t s) {
   const int ng = nt / 32;
-#define DT_GEMM_CASE(NG, MODE, ST) \
-  if (ng == NG && mode == MODE && stoch == ST) \
-    return launch_cfg<NG, 16, MODE, ST>(tmW, tmH, a, batch, ntiles, s);
-  DT_GEMM_CASE(1, EPI_EXPAND, false)
-  DT_GEMM_CASE(2, EPI_EXPAND, false)
-  DT_GEMM_CASE(1, EPI_EXPAND, true)
-  DT_GEMM_CASE(2, EPI_EXPAND, true)
-  DT_GEMM_CASE(1, EPI_ZDUMP, false)
-  DT_GEMM_CASE(2, EPI_ZDUMP, false)
-  DT_GEMM_CASE(1, EPI_QROWS, true)
-  DT_GEMM_CASE(2, EPI_QROWS, true)
+  a.n_ntiles = (a.Mcap + nt - 1) / nt;
+  if (a.ldo == 0) a.ldo = a.V;
+  if (ng == 8 && mode == EPI_EXPAND && a.L) return cudaErrorInvalidValue;  // no bias path
+  const int kmax = gemm_kmax(a.k);
+#define DT_GEMM_CASE(NG, MODE, ST, KM)                                                  \
+  if (ng == NG && mode == MODE && stoch == ST && (MODE != EPI_EXPAND || kmax == KM)) \
+    return launch_cfg<NG, MODE, ST, KM>(tmW, tmW2, tmH, a, batch, s);
+  DT_GEMM_CASE(1, EPI_EXPAND, false, 4)
+  DT_GEMM_CASE(1, EPI_EXPAND, false, 16)
+  DT_GEMM_CASE(2, EPI_EXPAND, false, 4)
+  DT_GEMM_CASE(2, EPI_EXPAND, false, 16)
+  DT_GEMM_CASE(8, EPI_EXPAND, false, 4)
+  DT_GEMM_CASE(8, EPI_EXPAND, false, 16)
+  DT_GEMM_CASE(1, EPI_EXPAND, true, 4)
+  DT_GEMM_CASE(1, EPI_EXPAND, true, 16)
+  DT_GEMM_CASE(2, EPI_EXPAND, true, 4)
+  DT_GEMM_CASE(2, EPI_EXPAND, true, 16)
+  DT_GEMM_CASE(1, EPI_ZDUMP, false, 4)
+  DT_GEMM_CASE(2, EPI_ZDUMP, false, 4)
+  DT_GEMM_CASE(8, EPI_ZDUMP, false, 4)
+  DT_GEMM_CASE(1, EPI_QROWS, true, 4)
+  DT_GEMM_CASE(2, EPI_QROWS, true, 4)
+  DT_GEMM_CASE(1, EPI_SWIGLU, false, 4)
+  DT_GEMM_CASE(2, EPI_SWIGLU, false, 4)
+  DT_GEMM_CASE(8, EPI_SWIGLU, false, 4)
 #undef DT_GEMM_CASE
   return cudaErrorInvalidValue;
 }

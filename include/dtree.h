@@ -129,6 +129,40 @@ dt_status dt_markov_logits(const void* d_block_logits, dt_dtype ldt,
                            dt_stream stream);
 size_t dt_markov_logits_workspace_bytes(int n_rows, int V, int r);
 
+/* ------------------------------------------------------------- TreeFlash --
+ * One TreeFlash draft-tree build (TreeFlash explainer, method sections 1-2)
+ * for `batch` requests, greedy (T = 0):
+ *   stage 1: S_i = the M best tokens of W_lm h_i, i = 1..gamma (ties to the
+ *            lower id): M unique tokens per depth;
+ *   stage 2: for depth 1 with the root as previous token, and for depth
+ *            i >= 2 with every t in S_{i-1}: 1 + (gamma-1) M evaluations of
+ *            h' = h_i + W_down(silu(W_gate x) * (W_up x)),
+ *            x = [rmsnorm(h_i) w_h :: rmsnorm(E[t]) w_e] (eps 1e-6),
+ *            q' = softmax(W_lm h');
+ *   select:  the best-first top-`budget` nodes by cumulative log q' (the
+ *            explainer names OPT-Tree; this reading takes the nodes of
+ *            highest path probability) under the order key desc, depth asc,
+ *            parent index asc, rank asc.  A node's candidates are the M best
+ *            tokens of its distribution; a node whose token is outside
+ *            S_depth was not evaluated and is a leaf.
+ * x, silu(g) * u and h' are rounded to bf16 where they feed the next GEMM.
+ * Inputs (device, bf16 unless noted): d_h [batch][gamma][D] drafter hidden
+ * states of the block; d_embed [V][D]; d_w_norm_h, d_w_norm_e [D] fp32;
+ * d_w_gate, d_w_up [Dff][2D]; d_w_down [D][Dff]; d_w_lm [V][D];
+ * d_root [batch] int32 (last committed token).  Base pointers 16-byte
+ * aligned.  Outputs: the dt_tree arrays with Nmax = budget (d_draft_q
+ * unused).  Limits: D and Dff multiples of 64, M <= 16, budget <= 64,
+ * gamma <= 64, batch <= 1024, V < 2^24. */
+size_t dt_treeflash_workspace_bytes(int batch, int gamma, int D, int Dff, int V, int M,
+                                    int budget);
+dt_status dt_treeflash_build(const uint16_t* d_h, const uint16_t* d_embed,
+                             const float* d_w_norm_h, const float* d_w_norm_e,
+                             const uint16_t* d_w_gate, const uint16_t* d_w_up,
+                             const uint16_t* d_w_down, const uint16_t* d_w_lm,
+                             const int32_t* d_root, int batch, int gamma, int D, int Dff,
+                             int V, int M, int budget, const dt_tree* out, void* ws,
+                             size_t ws_bytes, dt_stream stream);
+
 /* ---------------------------------------------------------- verify attn --
  * out[b][i][h] = sum_j softmax_j(scale * q[b][i][h] . k_j + mask) v_j over
  * the columns request b's row i may see (TreeSpark article, introduction:
@@ -224,8 +258,9 @@ typedef enum {
   DT_K_ACCEPT_WALK = 5,
   DT_K_ATTN = 6,
   DT_K_ATTN_COMBINE = 7,
-  DT_K_TOPK = 8,          /* one wave of softmax statistics + top-k per node  */
-  DT_K_OTHER = 9
+  DT_K_OTHER = 8,
+  DT_K_TF_LMHEAD = 9,     /* TreeFlash LM head + top-M epilogue               */
+  DT_K_TF_MLP = 10        /* TreeFlash SwiGLU / down projection               */
 } dt_kernel_kind;
 
 /* Profiling hook (measurement only; off by default).  While set, every kernel
