@@ -39,7 +39,11 @@ DESCS = {
                  "T=0.6 stochastic (Philox), verify 32q/8kv d=128 prefix 4096, batch 1"),
     "load_adaptive": ("load-adaptive batch: 64 requests, B=7, V=151936, per-request budget from "
                       "{chain, 8, 16, 32}, lambda 0.01, T=1.0, lognormal prefixes 512..8192"),
+    "treeflash": ("TreeFlash tree build: SwiGLU AR-approximator d=2560, d_ff=2560, bf16 LM head "
+                  "2560x151936, M=4, depth 16 (61 evaluations per request), budget B=16, "
+                  "batch 16, T=0"),
 }
+TF = dict(V=151936, D=2560, Dff=2560, gamma=16, M=4, budget=16, batch=16)
 
 
 def parse():
@@ -50,7 +54,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--copies", type=int, default=4)
     p.add_argument("--no-oracle", action="store_true", help="skip the cpu_baseline leg")
-    p.add_argument("--workload", default=WORKLOAD, choices=["qwen3_4b", "qwen3_8b", "load_adaptive"])
+    p.add_argument("--workload", default=WORKLOAD, choices=["qwen3_4b", "qwen3_8b", "load_adaptive", "treeflash"])
     return p.parse_args()
 
 
@@ -333,14 +337,14 @@ def run_ours(args):
                  "us_per_step": 1e3 * sum(v) / kprof} for nm, v in per_kind.items()}
 
     # ---- roofline of the dominant kernel (the Markov GEMM waves).  Per launch
-    # it must stream the whole Markov factor Bm [V][r] bf16 once, read the
-    # block-logit rows of the requests, the gathered node rows and write one
-    # fp32 row of scaled logits per expanded node.  `cols` = expanded nodes
-    # per wave, counted from the final trees (wasted expansions excluded).
+    # it must stream the whole Markov factor Bm [V][r] bf16 once, read one
+    # block-logit row per request and the gathered node rows; its outputs
+    # (per-CTA softmax statistics and top-k lists) are a few KB.  `cols` =
+    # expanded nodes per wave, counted from the final trees.
     pk, pk_kind = peaks()
     cols = inner / Bk
     lbytes = 2 if w.logit_dtype == "bf16" else 4
-    gemm_bytes = V * r * 2 + B * V * lbytes + cols * (V * 4 + r * 2)
+    gemm_bytes = V * r * 2 + B * V * lbytes + cols * r * 2
     gemm_flops = 2.0 * cols * V * r
     g_us = kern["markov_gemm"]["avg_us"]
     t_hbm = gemm_bytes / (pk["hbm_gbs"] * 1e9)
@@ -354,7 +358,7 @@ def run_ours(args):
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                 "unit": "GB/s"}
     roof.update({"frac": round(achieved / roof["peak"], 4), "peak_kind": pk_kind,
-                 "kernel": "markov_gemm (one wave: tcgen05 Markov-head GEMM, s-row epilogue)",
+                 "kernel": "markov_gemm (one wave: tcgen05 Markov-head GEMM + fused softmax/top-k epilogue)",
                  "algorithmic_bytes_per_launch": int(gemm_bytes),
                  "algorithmic_flops_per_launch": int(gemm_flops),
                  "nodes_per_wave": round(cols, 2),
@@ -436,6 +440,148 @@ def run_ours(args):
         print(json.dumps(out))
 
 
+def run_treeflash(args):
+    """TreeFlash build throughput (one GPU): dt_treeflash_build replayed from a graph."""
+    import ctypes
+    import torch
+    import draft_tree_construction_markov_b200 as dt
+    from gen import treeflash_inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    bf = torch.bfloat16
+    V, D, Dff, gamma, M, budget, B = (TF[x] for x in ("V", "D", "Dff", "gamma", "M", "budget", "batch"))
+    x = treeflash_inputs(rank, V=V, D=D, Dff=Dff, positions=gamma, batch=B)
+    cu = lambda a, t=None: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(t or torch.float32)
+    d = dict(h=cu(x["h"], bf), E=cu(x["E"], bf), wh=cu(x["w_norm_h"]), we=cu(x["w_norm_e"]),
+             gate=cu(x["W_gate"], bf), up=cu(x["W_up"], bf), down=cu(x["W_down"], bf),
+             lm=cu(x["W_lm"], bf), root=torch.from_numpy(x["root"]).to(dev))
+    tree = dt.Tree.empty(B, budget, V, stochastic=False, device=dev)
+    ws = dt.workspace(dt.treeflash_workspace_bytes(B, gamma, D, Dff, V, M, budget), dev)
+
+    def step():
+        dt.treeflash_build(d["h"], d["E"], d["wh"], d["we"], d["gate"], d["up"], d["down"],
+                           d["lm"], d["root"], M=M, budget=budget, out=tree, ws=ws)
+
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            step()
+    torch.cuda.synchronize()
+    assert dt.read_status(ws) == 0
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        step()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    value = args.steps / (ms / 1e3)
+    assert dt.read_status(ws) == 0
+
+    # per-kernel live timing through the library's event hook
+    kprof = min(args.steps, 20)
+    cap = 32 * kprof
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap)]
+    for e in evs:
+        e.record(stream)
+    torch.cuda.synchronize()
+    ev_arr = (ctypes.c_void_p * (2 * cap))(*[e.cuda_event for e in evs])
+    kinds = (ctypes.c_int32 * cap)()
+    count = ctypes.c_int32(0)
+    dt._lib.lib.dt_set_profile_events(ev_arr, kinds, cap, ctypes.byref(count))
+    with torch.cuda.stream(stream):
+        for _ in range(kprof):
+            step()
+    torch.cuda.synchronize()
+    dt._lib.lib.dt_set_profile_events(None, None, 0, None)
+    per_kind = {}
+    for i in range(count.value):
+        per_kind.setdefault(dt._lib.KERNEL_KINDS[kinds[i]], []).append(
+            evs[2 * i].elapsed_time(evs[2 * i + 1]))
+    kern = {nm: {"launches_per_step": len(v) / kprof, "avg_us": 1e3 * statistics.mean(v),
+                 "us_per_step": 1e3 * sum(v) / kprof} for nm, v in per_kind.items()}
+
+    # roofline: the two LM-head launches per step (stage 1 over the block rows,
+    # stage 2 over the approximator rows) are dense bf16 contractions
+    pk, pk_kind = peaks()
+    n1, n2 = B * gamma, B * (1 + (gamma - 1) * M)
+    lm_flops = 2.0 * (n1 + n2) * V * D
+    lm_us = kern["tf_lmhead"]["us_per_step"]
+    achieved = lm_flops / (lm_us * 1e-6) / 1e12
+    roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "peak_kind": pk_kind,
+            "kernel": "tf_lmhead (tcgen05 LM head + fused log-sum-exp/top-M epilogue, 2 launches/step)",
+            "algorithmic_flops_per_step": int(lm_flops), "traffic": None,
+            "us_per_step": round(lm_us, 2)}
+
+    # end to end: hidden states and roots from pinned host memory, tree back
+    h_h = torch.from_numpy(np.ascontiguousarray(x["h"])).to(bf).pin_memory()
+    h_r = torch.from_numpy(x["root"]).pin_memory()
+    o_tok = torch.empty(B, budget, dtype=torch.int32).pin_memory()
+    o_par = torch.empty(B, budget, dtype=torch.int32).pin_memory()
+    o_n = torch.empty(B, dtype=torch.int32).pin_memory()
+    ke = min(args.steps, 30)
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            d["h"].copy_(h_h, non_blocking=True)
+            d["root"].copy_(h_r, non_blocking=True)
+            step()
+            o_tok.copy_(tree.tokens, non_blocking=True)
+            o_par.copy_(tree.parents, non_blocking=True)
+            o_n.copy_(tree.n_nodes, non_blocking=True)
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e3.record(stream)
+    torch.cuda.synchronize()
+    e2e = {"value": round(ke / (e2.elapsed_time(e3) / 1e3), 2), "unit": "builds/s",
+           "h2d_bytes_per_step": int(h_h.numel() * 2 + h_r.numel() * 4),
+           "d2h_bytes_per_step": int((o_tok.numel() + o_par.numel() + o_n.numel()) * 4),
+           "steps": ke, "path": "python API (eager launches) + pinned H2D/D2H copies"}
+    out = {
+        "metric": "TreeFlash draft-tree builds/s (batch of 16 requests)", "value": round(value, 2),
+        "unit": "builds/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": DESCS["treeflash"], "l2": "LM head 778 MB > 126 MB L2 per step",
+                   "round": "CUDA graph", "request_builds_per_s": round(B * value, 1)},
+        "roofline": roof,
+        "kernels": {nm: {kk: round(vv, 3) for kk, vv in dd.items()} for nm, dd in kern.items()},
+        "gpu_launches": int(round(count.value / kprof * args.steps)),
+        "e2e": e2e, "clocks": clk,
+        "tree_nodes": int(tree.n_nodes.sum().item()),
+    }
+    if not args.no_oracle:
+        from oracle import treeflash as otf
+        t0 = time.time()
+        otf.treeflash_tree(x["h"][0], x["E"], int(x["root"][0]), M, budget, x["w_norm_h"],
+                           x["w_norm_e"], x["W_gate"], x["W_up"], x["W_down"], x["W_lm"],
+                           store=otf.bf16_rne)
+        el = time.time() - t0
+        out["cpu_baseline"] = {"value": round(1.0 / (B * el), 5), "unit": "builds/s",
+                               "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"1 of the 16 requests in {el:.1f} s (numpy fp64), "
+                                         "scaled to a batch of 16"}
+    print(json.dumps(out))
+
+
 def run_reference(args):
     """The oracle as the reference arm: each step is one CPU round of the workload."""
     rank, world, local = dist_env()
@@ -479,5 +625,7 @@ if __name__ == "__main__":
     a = parse()
     if a.impl == "reference":
         run_reference(a)
+    elif a.workload == "treeflash":
+        run_treeflash(a)
     else:
         run_ours(a)

@@ -56,12 +56,6 @@ cudaError_t ensure_smem_ptr(const void* kernel, size_t bytes) {
   return cudaSuccess;
 }
 
-// Rows of the block logits start on 16-byte boundaries (vector bias loads).
-static int l_vec_ok(const void* L, dt_dtype ldt, int V) {
-  if ((uintptr_t)L & 15) return 0;
-  return ldt == DT_BF16 ? (V % 8 == 0) : (V % 4 == 0);
-}
-
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -221,7 +215,6 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   memset(&g, 0, sizeof(g));
   g.L = d_block_logits;
   g.l_bf16 = ldt == DT_BF16;
-  g.l_vec = l_vec_ok(d_block_logits, ldt, V);
   g.Bk = Bk;
   g.V = V;
   g.r = r;

@@ -51,7 +51,6 @@ enum EpiMode { EPI_EXPAND = 0, EPI_ZDUMP = 1, EPI_QROWS = 2, EPI_SWIGLU = 3 };
 struct GemmArgs {
   const void* L;         // bias rows [batch][Bk][V] (block logits, residual) or NULL
   int l_bf16;
-  int l_vec;             // rows of L are 16-byte aligned (vector bias loads)
   int Bk, V, r, k;       // V: weight rows (vocabulary / features), r: inner dimension
   const Row* rows;       // GEMM columns
   const int32_t* n_rows; // device count of valid columns
@@ -59,6 +58,8 @@ struct GemmArgs {
   int n_vtiles;          // weight tiles (128 rows; SwiGLU: 64 features)
   int ncta_v;            // weight ranges (= partials per node)
   int n_ntiles;          // node tiles for Mcap columns (set by the launcher)
+  int bias_span;         // bias cache row length (set by the launcher; 0 = no cache)
+  int bias_rows;         // bias cache capacity in rows (set by the launcher)
   int Mcap;              // capacity of rows
   float temp;
   uint64_t seed;

@@ -22,10 +22,11 @@
 //  * EXPAND (the hot path of both trees): four warps per 32 node columns read
 //    the accumulator back with tcgen05.ld (each warp its 32-lane quadrant = 32
 //    vocabulary rows) and transpose each 32 x 32 block through shared memory,
-//    so every thread owns ONE node column and scans 32 consecutive vocabulary
-//    entries of it per tile.  Per column it fuses the block-logit bias
-//    (prefetched one tile ahead), the temperature, a batched max / sum-exp, a
-//    private top-k of s (ties to the lower token id) and, at T > 0, the
+//    so every thread owns one node column and scans consecutive vocabulary
+//    entries of it per tile (several lanes share a column when the block has
+//    few live columns).  Per column it fuses the block-logit bias (prefetched
+//    one tile ahead), the temperature, an online max / sum-exp, a private
+//    top-k of s (ties to the lower token id) and, at T > 0, the
 //    Gumbel-top-k of s + G (TreeSpark article, "lossless" section;
 //    Gumbel-top-k: Kool, van Hoof and Welling 2019), one Philox call per four
 //    consecutive tokens.  The CTA writes one partial result per node; a later
@@ -37,6 +38,7 @@
 //    the same features (lanes 64-127); the up quadrants hand their values to
 //    the gate quadrants through shared memory, which store silu(g) * u (bf16).
 #include "build.cuh"
+#include "merge.cuh"
 
 namespace dt {
 
@@ -74,10 +76,15 @@ struct ColMeta {
   int32_t valid;
   float lse;
   int32_t out_row;
+  int32_t bslot;     // row of the shared-memory bias cache (-1: not cached)
+  int32_t pad;
 };
 
+// Most distinct bias rows a CTA keeps in shared memory for its vocabulary range.
+constexpr int kBiasRowsMax = 32;
+
 template <int NG>
-static size_t gemm_epi_bytes(int mode, int kmax, bool stoch) {
+__host__ __device__ inline size_t gemm_epi_bytes(int mode, int kmax, bool stoch) {
   using S = GemmShape<NG>;
   const size_t tbuf = (size_t)S::kEpiWarps * 32 * kTLD * 4;
   if (mode == EPI_SWIGLU) return tbuf;
@@ -88,16 +95,24 @@ static size_t gemm_epi_bytes(int mode, int kmax, bool stoch) {
 }
 
 template <int NG>
-static size_t gemm_smem_bytes(int stages, int mode, int kmax, bool stoch) {
+static size_t gemm_smem_bytes(int stages, int mode, int kmax, bool stoch, size_t bias_bytes) {
   using S = GemmShape<NG>;
   size_t off = 1024;  // alignment slack
   off += (size_t)stages * S::kStageBytes;
   off += (size_t)(2 * stages + 2 * S::kAccBufs + 5) * 8;  // barriers
   off += 16;                                             // tmem slot + abort flag
   off = (off + 15) & ~(size_t)15;
-  off += (size_t)S::NT * sizeof(ColMeta);
+  off += (size_t)S::NT * sizeof(ColMeta) + 16 + kBiasRowsMax * 8;
   off += gemm_epi_bytes<NG>(mode, kmax, stoch);
+  off = (off + 15) & ~(size_t)15;
+  off += bias_bytes;
   return off;
+}
+
+// 16-byte global -> shared copy that does not block the thread.
+__device__ __forceinline__ void cp_async16_g2s(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
 }
 
 // Insert (v, id) into a register list sorted by value (descending) when ids
@@ -129,11 +144,6 @@ __device__ __forceinline__ float kth(const float (&L)[KMAX], int k) {
   for (int i = 1; i < KMAX; ++i)
     if (i == k - 1) t = L[i];
   return t;
-}
-
-// (v1, i1) ranks before (v2, i2): larger value first, then lower id.
-__device__ __forceinline__ bool ranks_before(float v1, int32_t i1, float v2, int32_t i2) {
-  return v1 > v2 || (v1 == v2 && i1 < i2);
 }
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
@@ -172,6 +182,13 @@ __device__ __forceinline__ void decode_bias(const uint4 (&raw)[8], int bf16, flo
   }
 }
 
+// 2^x with the hardware approximation (relative error below 2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float load_bias1(const void* L, int bf16, int64_t off) {
   return bf16 ? bf16_to_f32(__ldg((const uint16_t*)L + off)) : __ldg((const float*)L + off);
 }
@@ -204,13 +221,19 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // node tile fastest: the CTAs that share a weight range run side by side
   const int cx = blockIdx.x / a.n_ntiles, ny = blockIdx.x % a.n_ntiles;
-  // the node rows, their count and the gathered rows come from the previous kernel
-  pdl_wait();
-  const int M = min(*a.n_rows, a.Mcap);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && a.reset_count) *a.reset_count = 0;
-  pdl_launch_dependents();
-  if (ny * S::NT >= M) return;  // uniform over the CTA
-
+  // The first node tile has work whenever any node does: its CTAs set up and
+  // start streaming weights before the previous kernel finishes.  CTAs of
+  // later node tiles first check that they have columns at all.
+  const bool early = ny == 0;
+  int M = 0;
+  if (!early) {
+    pdl_wait();
+    M = min(*a.n_rows, a.Mcap);
+    if (ny * S::NT >= M) {
+      pdl_launch_dependents();
+      return;  // uniform over the CTA
+    }
+  }
   const int base = a.n_vtiles / a.ncta_v, extra = a.n_vtiles % a.ncta_v;
   const int t0 = cx * base + min(cx, extra);
   const int t1 = t0 + base + (cx < extra ? 1 : 0);
@@ -237,7 +260,16 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
   p = (uint8_t*)(((uintptr_t)p + 15) & ~(uintptr_t)15);
   ColMeta* meta = (ColMeta*)p;
   p += S::NT * sizeof(ColMeta);
+  int* n_bias = (int*)p;  // distinct cached bias rows (-1: cache not used)
+  p += 16;
+  int64_t* brow = (int64_t*)p;  // [kBiasRowsMax] element offsets of the cached rows
+  p += kBiasRowsMax * 8;
   float* tbuf = (float*)p;  // [kEpiWarps][32][kTLD]; EXPAND: then the quadrant partials
+  p += gemm_epi_bytes<NG>(MODE, KMAX, STOCH);
+  p = (uint8_t*)(((uintptr_t)p + 15) & ~(uintptr_t)15);
+  // [kBiasRows][bias_span] values of the distinct bias rows over this CTA's
+  // vocabulary range (same element type as L)
+  uint8_t* bias_cache = p;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -261,6 +293,44 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
     if (MODE == EPI_SWIGLU) prefetch_tmap(&tmW2);
     prefetch_tmap(&tmH);
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::kTmemCols);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // The weight tiles do not depend on the previous kernel: the first stages
+  // start streaming while it finishes (each stage's barrier also waits for
+  // its node-row box, issued below once those rows exist).
+  const int total = (t1 - t0) * KC;
+  const int npre = early ? min(stages, total) : 0;
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < npre; ++i) {
+      const int t = t0 + i / KC, kc = i % KC;
+      uint8_t* sa = stage_mem + (size_t)i * S::kStageBytes;
+      mbar_expect_tx(&full[i], S::kABytes);
+      if (MODE == EPI_SWIGLU) {
+        // 64 gate rows, then the 64 up rows of the same features
+        tma_load_2d(sa, &tmW, &full[i], kc * 64, t * 64);
+        tma_load_2d(sa + S::kABytes / 2, &tmW2, &full[i], kc * 64, t * 64);
+      } else {
+        tma_load_2d(sa, &tmW, &full[i], kc * 64, t * kTileV);
+      }
+    }
+  }
+
+  // the node rows, their count and the gathered rows come from the previous kernel
+  if (early) {
+    pdl_wait();
+    M = min(*a.n_rows, a.Mcap);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && a.reset_count) *a.reset_count = 0;
+  pdl_launch_dependents();
+  const bool active = ny * S::NT < M;  // uniform over the CTA
+  // a CTA without node columns only completes the copies it started
+  const int t_end = active ? t1 : t0;
   for (int c = threadIdx.x; c < S::NT; c += blockDim.x) {
     const int row = ny * S::NT + c;
     ColMeta cm;
@@ -270,6 +340,8 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
     cm.b = 0;
     cm.lse = 0.f;
     cm.out_row = 0;
+    cm.bslot = -1;
+    cm.pad = 0;
     if (row < M) {
       const Row r = a.rows[row];
       if (r.b >= 0) {
@@ -288,47 +360,82 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
     }
     meta[c] = cm;
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, S::kTmemCols);
-    tc_fence_before();
-  }
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
+  // The expansion epilogue reads its bias rows from shared memory: global
+  // loads issued during the weight stream wait behind it for microseconds.
+  if (MODE == EPI_EXPAND) {
+    if (threadIdx.x == 0) {
+      int nb = 0;
+      bool ok = a.bias_span > 0 && a.bias_rows > 0 && a.L != nullptr && active;
+      for (int c = 0; c < S::NT && ok; ++c) {
+        if (!meta[c].valid) continue;
+        int u = -1;
+        for (int i = 0; i < nb; ++i)
+          if (brow[i] == meta[c].bias_off) u = i;
+        if (u < 0) {
+          if (nb == a.bias_rows) {
+            ok = false;
+            break;
+          }
+          brow[nb] = meta[c].bias_off;
+          u = nb++;
+        }
+        meta[c].bslot = u;
+      }
+      *n_bias = ok ? nb : -1;
+    }
+    __syncthreads();
+    const int nb = *n_bias;
+    if (warp >= 2 && nb > 0) {
+      // every 16-byte piece of [t0 * 128, min(t1 * 128, V)) of each distinct row
+      const int esz = a.l_bf16 ? 2 : 4;
+      const int x0 = t0 * kTileV;
+      const int nx = min(t1 * kTileV, a.V) - x0;
+      const int npieces = (nx * esz + 15) / 16;
+      for (int u = 0; u < nb; ++u) {
+        const uint8_t* src = (const uint8_t*)a.L + (brow[u] + x0) * esz;
+        uint8_t* dst = bias_cache + (size_t)u * a.bias_span * esz;
+        for (int i = threadIdx.x - 64; i < npieces; i += S::kEpiWarps * 32)
+          cp_async16_g2s(dst + (size_t)i * 16, src + (size_t)i * 16);
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
       bool ok = true;
       uint32_t issued = 0, last_parity = 0;  // per stage: issued at least once, parity of last issue
-      for (int t = t0; t < t1 && ok; ++t) {
-        for (int kc = 0; kc < KC; ++kc) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, a.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sa = stage_mem + (size_t)stage * S::kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
-          if (MODE == EPI_SWIGLU) {
-            // 64 gate rows, then the 64 up rows of the same features
-            tma_load_2d(sa, &tmW, &full[stage], kc * 64, t * 64);
-            tma_load_2d(sa + S::kABytes / 2, &tmW2, &full[stage], kc * 64, t * 64);
-          } else {
-            tma_load_2d(sa, &tmW, &full[stage], kc * 64, t * kTileV);
-          }
-          tma_load_2d(sa + S::kABytes, &tmH, &full[stage], kc * 64, ny * S::NT);
-          issued |= 1u << stage;
-          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == stages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
+      for (int i = 0; i < npre; ++i) {
+        uint8_t* sa = stage_mem + (size_t)i * S::kStageBytes;
+        mbar_arrive_expect_tx(&full[i], S::kBBytes);
+        tma_load_2d(sa + S::kABytes, &tmH, &full[i], (i % KC) * 64, ny * S::NT);
+        issued |= 1u << i;
       }
-      if (!ok) {
-        // let the copies already in flight land (bounded) before the CTA exits
+      const int n_all = active ? total : npre;
+      for (int i = npre; i < n_all; ++i) {
+        const int stage = i % stages;
+        const uint32_t phase = (uint32_t)(i / stages) & 1u;
+        const int t = t0 + i / KC, kc = i % KC;
+        if (!mbar_wait(&empty[stage], phase ^ 1, a.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = stage_mem + (size_t)stage * S::kStageBytes;
+        mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+        if (MODE == EPI_SWIGLU) {
+          tma_load_2d(sa, &tmW, &full[stage], kc * 64, t * 64);
+          tma_load_2d(sa + S::kABytes / 2, &tmW2, &full[stage], kc * 64, t * 64);
+        } else {
+          tma_load_2d(sa, &tmW, &full[stage], kc * 64, t * kTileV);
+        }
+        tma_load_2d(sa + S::kABytes, &tmH, &full[stage], kc * 64, ny * S::NT);
+        issued |= 1u << stage;
+        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+      }
+      if (!ok || !active) {
+        // let the copies in flight land (bounded) before the CTA exits
         const uint64_t t_start = globaltimer_ns();
         for (int st = 0; st < stages; ++st) {
           if (!((issued >> st) & 1)) continue;
@@ -347,7 +454,7 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
       int ab = 0;
       uint32_t aphase = 0;
       bool ok = true;
-      for (int t = t0; t < t1 && ok; ++t) {
+      for (int t = t0; t < t_end && ok; ++t) {
         if (!mbar_wait(&tempty[ab], aphase ^ 1, a.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(ab * S::NT);
@@ -389,7 +496,7 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
     const int eg = e >> 2;   // column group served by this warp
     int ab = 0;
     uint32_t aphase = 0;
-    for (int t = t0; t < t1; ++t) {
+    for (int t = t0; t < t_end; ++t) {
       const int x = t * kTileV + 32 * q + lane;
       if (!mbar_wait(&tfull[ab], aphase, a.status, abort_flag)) break;
       tc_fence_after();
@@ -442,7 +549,7 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
     uint32_t aphase = 0;
     uint32_t xn = 0;  // exchanges so far (phase parity)
     bool ok = true;
-    for (int t = t0; t < t1 && ok; ++t) {
+    for (int t = t0; t < t_end && ok; ++t) {
       const int f = t * 64 + 32 * (q & 1) + lane;  // feature of this lane
       if (!mbar_wait(&tfull[ab], aphase, a.status, abort_flag)) break;
       tc_fence_after();
@@ -490,6 +597,11 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
     }
   } else {
     // --------------------------------------------- expansion epilogue (columns)
+    // Each 32 x 32 accumulator block (32 vocabulary rows of quadrant q, 32
+    // node columns) is transposed through the warp's buffer so that lane c
+    // owns column c and holds its 32 consecutive rows.  The arithmetic per
+    // block is branch-free (tree max and sum, independent 2^x); the top-k
+    // lists are only touched when the block's maximum beats the entry bar.
     const int e = warp - 2;
     const int q = warp & 3;  // TMEM lane quadrant accessible to this warp
     const int eg = e >> 2;   // first column group of this warp
@@ -517,19 +629,26 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
         I2[j][i] = 0x7fffffff;
       }
     }
-    // bias rows (one column group per thread only): requested one tile ahead
-    const bool has_bias = S::CPT == 1 && a.L != nullptr;
-    const bool vec = a.l_vec != 0;
+    // bias rows: from the shared-memory cache when it holds them all, else
+    // (one column group per thread only) global loads one tile ahead
+    const int nbc = *n_bias;
+    const bool cached = nbc > 0;
+    if (cached) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      named_bar(1, S::kEpiWarps * 32);
+    }
+    const bool ldg_bias = S::CPT == 1 && a.L != nullptr && !cached;
+    const bool vec = (a.l_bf16 ? (a.V % 8 == 0) : (a.V % 4 == 0)) && ((uintptr_t)a.L % 16 == 0);
     uint4 raw[8];
     bool raw_ok = false;
-    if (has_bias) {
+    if (ldg_bias) {
       const int xq = t0 * kTileV + 32 * q;
-      raw_ok = mc[0].valid && vec && xq + 32 <= a.V && t0 < t1;
+      raw_ok = mc[0].valid && vec && xq + 32 <= a.V && t0 < t_end;
       if (raw_ok) load_bias_raw(a.L, a.l_bf16, mc[0].bias_off + xq, raw);
     }
     int ab = 0;
     uint32_t aphase = 0;
-    for (int t = t0; t < t1; ++t) {
+    for (int t = t0; t < t_end; ++t) {
       if (!mbar_wait(&tfull[ab], aphase, a.status, abort_flag)) break;
       tc_fence_after();
       const int xq = t * kTileV + 32 * q;  // first vocabulary row of this quadrant
@@ -546,14 +665,14 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
         }
         float bias[32];
         bool had_raw = false;
-        if (has_bias) {
+        if (ldg_bias) {
           if (raw_ok) decode_bias(raw, a.l_bf16, bias);
           had_raw = raw_ok;
           const int xn = xq + kTileV;
-          raw_ok = mc[0].valid && vec && t + 1 < t1 && xn + 32 <= a.V;
+          raw_ok = mc[0].valid && vec && t + 1 < t_end && xn + 32 <= a.V;
           if (raw_ok) load_bias_raw(a.L, a.l_bf16, mc[0].bias_off + xn, raw);
         }
-        // transpose 32 rows x 32 columns: thread `lane` takes column grp*32+lane
+        // transpose 32 rows x 32 columns: lane takes column grp*32+lane
 #pragma unroll
         for (int i = 0; i < 32; ++i) tb[lane * kTLD + i] = acc[i];
         __syncwarp();
@@ -561,13 +680,35 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
         for (int i = 0; i < 32; ++i) acc[i] = tb[i * kTLD + lane];
         __syncwarp();
         if (!mc[j].valid || nv <= 0) continue;
-        if (!has_bias) {
+        if (cached) {
+          // 32 consecutive values of this column's bias row (16-byte reads)
+          const int xo = xq - t0 * kTileV;
+          if (nv == 32) {
+            uint4 cr[8];
+            const uint4* src = (const uint4*)(bias_cache + ((size_t)mc[j].bslot * a.bias_span + xo) *
+                                                               (a.l_bf16 ? 2 : 4));
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              if (c < 4 || !a.l_bf16) cr[c] = src[c];
+            decode_bias(cr, a.l_bf16, bias);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              bias[i] = i < nv ? (a.l_bf16 ? bf16_to_f32(((const uint16_t*)bias_cache)[
+                                                 (size_t)mc[j].bslot * a.bias_span + xo + i])
+                                           : ((const float*)bias_cache)[
+                                                 (size_t)mc[j].bslot * a.bias_span + xo + i])
+                               : 0.f;
+          }
+        } else if (ldg_bias) {
+          if (!had_raw) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              bias[i] = i < nv ? load_bias1(a.L, a.l_bf16, mc[j].bias_off + xq + i) : 0.f;
+          }
+        } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) bias[i] = 0.f;
-        } else if (!had_raw) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            bias[i] = i < nv ? load_bias1(a.L, a.l_bf16, mc[j].bias_off + xq + i) : 0.f;
         }
         float s[32];
 #pragma unroll
@@ -575,47 +716,61 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
           const float z = acc[i] + bias[i];
           s[i] = i < nv ? (STOCH ? __fdiv_rn(z, temp) : z) : -INFINITY;
         }
-        // log-sum-exp, batched over the 32 values
-        float mt = s[0];
+        // log-sum-exp of the block: tree max, independent 2^x, tree sum
+        float mx[16];
 #pragma unroll
-        for (int i = 1; i < 32; ++i) mt = fmaxf(mt, s[i]);
-        float st = 0.f;
+        for (int i = 0; i < 16; ++i) mx[i] = fmaxf(s[i], s[i + 16]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) st += exp2f((s[i] - mt) * kLog2e);
+        for (int w = 8; w; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+        const float mt = mx[0];
+        float ex[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ex[i] = ex2_approx((s[i] - mt) * kLog2e);
+#pragma unroll
+        for (int w = 16; w; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) ex[i] += ex[i + w];
+        const float st = ex[0];
         if (mt > m[j]) {
-          ssum[j] = ssum[j] * exp2f((m[j] - mt) * kLog2e) + st;
+          ssum[j] = ssum[j] * ex2_approx((m[j] - mt) * kLog2e) + st;
           m[j] = mt;
         } else {
-          ssum[j] += st * exp2f((mt - m[j]) * kLog2e);
+          ssum[j] += st * ex2_approx((mt - m[j]) * kLog2e);
         }
         // top-k of s (values arrive in increasing token order)
+        if (mt > thr[j]) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (s[i] > thr[j]) {
-            topk_insert<KMAX>(L1[j], I1[j], s[i], xq + i);
-            thr[j] = kth<KMAX>(L1[j], k);
+          for (int i = 0; i < 32; ++i) {
+            if (s[i] > thr[j]) {
+              topk_insert<KMAX>(L1[j], I1[j], s[i], xq + i);
+              thr[j] = kth<KMAX>(L1[j], k);
+            }
           }
         }
         if constexpr (STOCH) {
           // Gumbel keys; four consecutive tokens share one Philox counter
+          if (mt + kGumbelMax > gthr[j]) {
 #pragma unroll
-          for (int gi = 0; gi < 8; ++gi) {
-            const float smax =
-                fmaxf(fmaxf(s[4 * gi], s[4 * gi + 1]), fmaxf(s[4 * gi + 2], s[4 * gi + 3]));
-            if (!(smax + kGumbelMax > gthr[j])) continue;
-            const uint32_t x4 = (uint32_t)(xq + 4 * gi);
-            const U4 o =
-                philox10(U4{(x4 >> 2) | ((uint32_t)mc[j].b << 18), mc[j].c1, mc[j].c2, a.offset},
-                         (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
-            const uint32_t wds[4] = {o.x, o.y, o.z, o.w};
+            for (int gi = 0; gi < 8; ++gi) {
+              const float smax =
+                  fmaxf(fmaxf(s[4 * gi], s[4 * gi + 1]), fmaxf(s[4 * gi + 2], s[4 * gi + 3]));
+              if (!(smax + kGumbelMax > gthr[j])) continue;
+              const uint32_t x4 = (uint32_t)(xq + 4 * gi);
+              const U4 o = philox10(
+                  U4{(x4 >> 2) | ((uint32_t)mc[j].b << 18), mc[j].c1, mc[j].c2, a.offset},
+                  (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
+              const uint32_t wds[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              const int i = 4 * gi + jj;
-              if (i >= nv) continue;
-              const float gk = s[i] + (-logf(-logf(u23(wds[jj]))));
-              if (gk > gthr[j]) {
-                topk_insert<KMAX>(L2[j], I2[j], gk, xq + i);
-                gthr[j] = kth<KMAX>(L2[j], k);
+              for (int jj = 0; jj < 4; ++jj) {
+                const int i = 4 * gi + jj;
+                if (i >= nv) continue;
+                const float gk = s[i] + (-logf(-logf(u23(wds[jj]))));
+                if (gk > gthr[j]) {
+                  topk_insert<KMAX>(L2[j], I2[j], gk, xq + i);
+                  gthr[j] = kth<KMAX>(L2[j], k);
+                }
               }
             }
           }
@@ -680,7 +835,7 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
             if (hw >= k) continue;
             const float v = LV[(w * S::NT + c) * KMAX + hw];
             const int32_t id = LI[(w * S::NT + c) * KMAX + hw];
-            if (bw < 0 || ranks_before(v, id, bv, bi)) {
+            if (bw < 0 || ranks_first(v, id, bv, bi)) {
               bw = w;
               bv = v;
               bi = id;
@@ -742,11 +897,31 @@ static cudaError_t launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmW2,
                               const CUtensorMap& tmH, GemmArgs a, int batch, cudaStream_t s) {
   using SH = GemmShape<NG>;
   auto kern = markov_gemm_kernel<NG, MODE, STOCH, KMAX>;
-  // the deepest pipeline that fits in 220 KB of shared memory
+  // bias cache: the longest vocabulary range of a CTA, padded to 16 bytes;
+  // only when 16-byte copies of the rows are aligned
+  size_t bias_bytes = 0;
+  a.bias_span = 0;
+  a.bias_rows = 0;
+  if (MODE == EPI_EXPAND && a.L) {
+    const int esz = a.l_bf16 ? 2 : 4;
+    const bool aligned = ((uintptr_t)a.L % 16 == 0) && ((size_t)a.V * esz) % 16 == 0;
+    const int span = ((a.n_vtiles + a.ncta_v - 1) / a.ncta_v) * 128;
+    // distinct rows a node tile can need: one per (request, depth), at most NT
+    const int rows = std::min(std::min(SH::NT, kBiasRowsMax), batch * a.Bk);
+    const size_t bytes = (size_t)rows * span * esz;
+    if (aligned && bytes <= 80 * 1024) {
+      a.bias_span = span;
+      a.bias_rows = rows;
+      bias_bytes = bytes;
+    }
+  }
+  // the deepest pipeline that fits in 200 KB of shared memory, which leaves room
+  // on each SM for a small kernel of the wave loop running alongside
   int stages = 10;
-  while (stages > 2 && gemm_smem_bytes<NG>(stages, MODE, KMAX, STOCH) > 220 * 1024) --stages;
+  while (stages > 2 && gemm_smem_bytes<NG>(stages, MODE, KMAX, STOCH, bias_bytes) > 200 * 1024)
+    --stages;
   a.stages = stages;
-  const size_t smem = gemm_smem_bytes<NG>(stages, MODE, KMAX, STOCH);
+  const size_t smem = gemm_smem_bytes<NG>(stages, MODE, KMAX, STOCH, bias_bytes);
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.ncta_v * a.n_ntiles);

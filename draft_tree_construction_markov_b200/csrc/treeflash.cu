@@ -92,15 +92,44 @@ __global__ void tf_merge_kernel(const float2* pstats, const float* plv, const in
                     top_i + (size_t)row * M);
 }
 
-// Sum of squares of a bf16 row of length D (D % 256 == 0 not required), one warp.
+// 1 / rms of a bf16 row of length D (a multiple of 64), one warp, 16-byte loads.
 __device__ __forceinline__ float row_inv_rms(const uint16_t* x, int D, int lane) {
   float ss = 0.f;
-  for (int i = lane; i < D; i += 32) {
-    const float v = bf16_to_f32(x[i]);
-    ss = fmaf(v, v, ss);
+  const uint4* v = (const uint4*)x;
+  for (int i = lane; i < D / 8; i += 32) {
+    const uint4 u = v[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float lo = __uint_as_float(w[h] << 16), hi = __uint_as_float(w[h] & 0xFFFF0000u);
+      ss = fmaf(lo, lo, ss);
+      ss = fmaf(hi, hi, ss);
+    }
   }
   ss = warp_sum(ss);
   return rsqrtf(ss / (float)D + kRmsEps);
+}
+
+// dst[0..D) = bf16(src * inv * w), 8 elements per 16-byte access.
+__device__ __forceinline__ void row_norm_store(const uint16_t* src, const float* w, float inv,
+                                               uint16_t* dst, int D, int lane) {
+  const uint4* s4 = (const uint4*)src;
+  const float4* w4 = (const float4*)w;
+  uint4* d4 = (uint4*)dst;
+  for (int i = lane; i < D / 8; i += 32) {
+    const uint4 u = s4[i];
+    const float4 wa = w4[2 * i], wb = w4[2 * i + 1];
+    const float ww[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+    const uint32_t in[4] = {u.x, u.y, u.z, u.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float lo = __uint_as_float(in[h] << 16) * inv * ww[2 * h];
+      const float hi = __uint_as_float(in[h] & 0xFFFF0000u) * inv * ww[2 * h + 1];
+      out[h] = (uint32_t)to_bf16(lo) | ((uint32_t)to_bf16(hi) << 16);
+    }
+    d4[i] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
 }
 
 // One warp per evaluation row: its Row, and x = [rmsnorm(h_d) :: rmsnorm(E[t])].
@@ -130,10 +159,8 @@ __global__ void tf_prep_kernel(const uint16_t* h, const uint16_t* E, const float
   const float ih = row_inv_rms(hr, D, lane);
   const float ie = row_inv_rms(er, D, lane);
   uint16_t* xr = X + (size_t)e * 2 * D;
-  for (int i = lane; i < D; i += 32) {
-    xr[i] = to_bf16(bf16_to_f32(hr[i]) * ih * w_h[i]);
-    xr[D + i] = to_bf16(bf16_to_f32(er[i]) * ie * w_e[i]);
-  }
+  row_norm_store(hr, w_h, ih, xr, D, lane);
+  row_norm_store(er, w_e, ie, xr + D, D, lane);
   if (lane == 0) {
     Row r;
     r.b = b;
