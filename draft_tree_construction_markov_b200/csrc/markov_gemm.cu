@@ -361,9 +361,9 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
     meta[c] = cm;
   }
   __syncthreads();
-  // The expansion epilogue reads its bias rows from shared memory: global
-  // loads issued during the weight stream wait behind it for microseconds.
-  if (MODE == EPI_EXPAND) {
+  // The epilogues read their bias rows from shared memory: global loads
+  // issued during the weight stream wait behind it for microseconds.
+  if (MODE != EPI_SWIGLU) {
     if (threadIdx.x == 0) {
       int nb = 0;
       bool ok = a.bias_span > 0 && a.bias_rows > 0 && a.L != nullptr && active;
@@ -496,6 +496,11 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
     const int eg = e >> 2;   // column group served by this warp
     int ab = 0;
     uint32_t aphase = 0;
+    const bool cached = *n_bias > 0;
+    if (cached) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      named_bar(1, S::kEpiWarps * 32);
+    }
     for (int t = t0; t < t_end; ++t) {
       const int x = t * kTileV + 32 * q + lane;
       if (!mbar_wait(&tfull[ab], aphase, a.status, abort_flag)) break;
@@ -515,7 +520,14 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
         for (int i = 0; i < 32; ++i) {
           const ColMeta& cm = meta[grp * 32 + i];
           if (!cm.valid) continue;  // warp-uniform
-          const float bias = a.L ? load_bias1(a.L, a.l_bf16, cm.bias_off + x) : 0.f;
+          float bias = 0.f;
+          if (cached) {
+            const size_t ci = (size_t)cm.bslot * a.bias_span + (x - t0 * kTileV);
+            bias = a.l_bf16 ? bf16_to_f32(((const uint16_t*)bias_cache)[ci])
+                            : ((const float*)bias_cache)[ci];
+          } else if (a.L) {
+            bias = load_bias1(a.L, a.l_bf16, cm.bias_off + x);
+          }
           const float z = acc[i] + bias;
           if (MODE == EPI_ZDUMP) {
             if (a.out_bf16)
@@ -902,7 +914,7 @@ static cudaError_t launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmW2,
   size_t bias_bytes = 0;
   a.bias_span = 0;
   a.bias_rows = 0;
-  if (MODE == EPI_EXPAND && a.L) {
+  if (MODE != EPI_SWIGLU && a.L) {
     const int esz = a.l_bf16 ? 2 : 4;
     const bool aligned = ((uintptr_t)a.L % 16 == 0) && ((size_t)a.V * esz) % 16 == 0;
     const int span = ((a.n_vtiles + a.ncta_v - 1) / a.ncta_v) * 128;

@@ -75,10 +75,34 @@ __device__ __forceinline__ void merge_lists(const float* PV, const int32_t* PI, 
         pi[j][i] = in ? __ldcg(PI + (size_t)c * k + i) : 0x7fffffff;
       }
     }
+    // entry bar: the best kb-th entry of any partial.  Its partial alone holds
+    // kb entries at or above it, so nothing below it can be among the kb best.
+    float bv = -INFINITY;
+    int32_t bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < JP; ++j) {
+      float v;
+      int32_t id;
+      list_entry<KMAX>(pv[j], pi[j], kb - 1, v, id);
+      if (ranks_first(v, id, bv, bi)) {
+        bv = v;
+        bi = id;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ranks_first(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
 #pragma unroll
     for (int j = 0; j < JP; ++j) {
 #pragma unroll
       for (int i = 0; i < KMAX; ++i) {
+        if (ranks_first(bv, bi, pv[j][i], pi[j][i])) break;  // lists are sorted
         float kv;
         int32_t ki;
         list_entry<KMAX>(L, I, kb - 1, kv, ki);
