@@ -66,6 +66,21 @@ def dist_env():
 
 
 # ------------------------------------------------------------------ oracle --
+def max_over_ranks(ms, world, device):
+    """Slowest rank's time (ms): every rank joins the same all-reduce."""
+    import torch
+    t = torch.tensor([float(ms)], device=device)
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms_max):
+    """Whole-job units per second: every rank's units over the slowest rank's time."""
+    return world * units_per_rank / (ms_max / 1e3)
+
+
 def oracle_round(w, o_inputs):
     """One round of the CPU oracle on the bench workload (build, verify, accept)."""
     from gen import attention_inputs, target_rows
@@ -302,12 +317,8 @@ def run_ours(args):
     barrier()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    ms_t = torch.tensor([ms], device=dev)
-    if world > 1:
-        import torch.distributed as tdist
-        tdist.all_reduce(ms_t, op=tdist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
-    value = world * args.steps / (ms_max / 1e3)
+    ms_max = max_over_ranks(ms, world, dev)
+    value = job_throughput(args.steps, world, ms_max)
     for wsx in (ws_b, ws_v, ws_a):
         assert dt.read_status(wsx) == 0
 
@@ -401,11 +412,8 @@ def run_ours(args):
         e3.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms_e = torch.tensor([e2.elapsed_time(e3)], device=dev)
-    if world > 1:
-        import torch.distributed as tdist
-        tdist.all_reduce(ms_e, op=tdist.ReduceOp.MAX)
-    e2e = {"value": round(world * ke / (float(ms_e.item()) / 1e3), 1), "unit": UNIT,
+    ms_e = max_over_ranks(e2.elapsed_time(e3), world, dev)
+    e2e = {"value": round(job_throughput(ke, world, ms_e), 1), "unit": UNIT,
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": ke,
            "path": "python API (eager launches) + pinned H2D/D2H copies on the stream"}
 

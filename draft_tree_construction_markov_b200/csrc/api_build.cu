@@ -9,6 +9,7 @@ namespace dt {
 bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows,
                            uint32_t box_rows);
 int gemm_node_tile(int max_cols);
+bool gemm_can_gather(int r, int nt);
 cudaError_t launch_markov_gemm(int mode, bool stoch, const CUtensorMap& tmW,
                                const CUtensorMap& tmW2, const CUtensorMap& tmH, GemmArgs a,
                                int batch, int nt, cudaStream_t s);
@@ -89,7 +90,7 @@ struct BuildLayout {
   uint16_t* H;
   uint16_t* Hm;
   float2* pstats;  // [Mcap][ncta_v] per-CTA partials of the wave GEMM
-  float* plv;      // [Mcap][ncta_v][k]
+  float* plv;      // [Mcap][k][ncta_v]
   int32_t* pli;
   float* pgv;
   int32_t* pgi;
@@ -185,8 +186,11 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   memset(&f, 0, sizeof(f));
   f.mat_rows = L.mat_rows;
   f.mat_count = L.counts + 2;
-  f.H = L.H;
-  f.Hm = L.Hm;
+  // the GEMM gathers its node rows A[token] itself when they fit in shared
+  // memory; otherwise the frontier writes them to H / Hm for TMA
+  const bool gather = gemm_can_gather(r, L.nt);
+  f.H = gather ? nullptr : L.H;
+  f.Hm = gather ? nullptr : L.Hm;
   f.A = d_markov_a;
   f.req = L.req;
   f.lists = L.lists;
@@ -215,6 +219,7 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   memset(&g, 0, sizeof(g));
   g.L = d_block_logits;
   g.l_bf16 = ldt == DT_BF16;
+  g.gatherA = gather ? d_markov_a : nullptr;
   g.Bk = Bk;
   g.V = V;
   g.r = r;

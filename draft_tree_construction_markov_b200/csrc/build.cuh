@@ -60,16 +60,18 @@ struct GemmArgs {
   int n_ntiles;          // node tiles for Mcap columns (set by the launcher)
   int bias_span;         // bias cache row length (set by the launcher; 0 = no cache)
   int bias_rows;         // bias cache capacity in rows (set by the launcher)
+  const uint16_t* gatherA;  // [V][r]: gather B rows A[token] in the kernel (NULL: TMA from H)
   int Mcap;              // capacity of rows
   float temp;
   uint64_t seed;
   uint32_t offset;
-  // expand: one partial per (node row, CTA), index row * ncta_v + cta
+  // expand: one partial per (node row, CTA): statistics at row * ncta_v + cta,
+  // list entry i at (row * k + i) * ncta_v + cta
   float2* pstats;        // (max, sum exp(s - max)) of the CTA's vocabulary range
-  float* plv;            // [k] top-k values of s, best first (ties: lower token)
-  int32_t* pli;          // [k] their tokens
-  float* pgv;            // [k] Gumbel-top-k keys (T > 0)
-  int32_t* pgi;          // [k] their tokens
+  float* plv;            // top-k values of s, best first (ties: lower token)
+  int32_t* pli;          // their tokens
+  float* pgv;            // Gumbel-top-k keys (T > 0)
+  int32_t* pgi;          // their tokens
   // zdump: z, [aux][ldo] (fp32, or bf16 if out_bf16); qrows: q = exp(s - lse),
   // [b][Nmax+1][ldo] with row aux; swiglu: silu(gate) * up, bf16 [aux][ldo]
   float* out;
@@ -87,8 +89,8 @@ struct FrontierArgs {
   int32_t* next_count;
   Row* mat_rows;         // rows whose draft distribution is materialised (T > 0)
   int32_t* mat_count;
-  uint16_t* H;           // gathered Markov rows of the next wave [Mcap][r]
-  uint16_t* Hm;          // gathered Markov rows of mat_rows
+  uint16_t* H;           // gathered Markov rows of the next wave [Mcap][r] (NULL: the GEMM gathers)
+  uint16_t* Hm;          // gathered Markov rows of mat_rows (NULL: the GEMM gathers)
   const uint16_t* A;     // [V][r]
   ReqState* req;
   Cand* lists;           // [batch][Nmax]

@@ -44,6 +44,8 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
   __shared__ int s_cnt[4];        // kept nodes, next-wave base, rows scheduled, q-row base
   __shared__ int16_t s_pos[64];   // position among the scheduled (or q-row) nodes, -1 if none
   __shared__ int32_t s_par[64];
+  __shared__ float s_mv[kWarps][32];  // per-warp scratch of the partial merge
+  __shared__ int32_t s_mi[kWarps][32];
   if (tid == 0) st = f.req[b];  // written by the previous frontier step (two kernels back)
   __syncthreads();
   if (st.done) {
@@ -66,26 +68,27 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
   if (tid < 4) s_cnt[tid] = 0;
   // the per-CTA partials come from the wave GEMM launched just before
   pdl_wait();
-  pdl_launch_dependents();
 
   // 1. merge each expanded node's partials: its log-sum-exp and its kb best
   // (T = 0) or sampled (T > 0, Gumbel-top-k) children, one warp per node
   for (int e = warp; e < rows_n; e += kWarps) {
     const size_t prow = (size_t)(st.row_base + e) * f.ncta;
-    const float lse = merge_lse(f.pstats + prow, f.ncta, lane);
     // values of the k best (order statistics of s); tokens of the best (T = 0)
     // or of the Gumbel sample (T > 0)
     const bool stoch = f.temp > 0.f;
-    merge_lists<KMAX>(f.plv + prow * k, f.pli + prow * k, f.ncta, k, kb, lane, r_lq + e * k,
-                      stoch ? nullptr : r_tok + e * k);
-    if (stoch)
-      merge_lists<KMAX>(f.pgv + prow * k, f.pgi + prow * k, f.ncta, k, kb, lane, nullptr,
-                        r_tok + e * k);
+    const float lse = merge_node<KMAX>(f.pstats + prow, f.plv + prow * k, f.pli + prow * k,
+                                       stoch ? f.pgv + prow * k : nullptr,
+                                       stoch ? f.pgi + prow * k : nullptr, f.ncta, k, kb, lane,
+                                       r_lq + e * k, stoch ? nullptr : r_tok + e * k,
+                                       stoch ? r_tok + e * k : nullptr, s_mv[warp], s_mi[warp]);
     __syncwarp();
     if (lane == 0) r_lse[e] = lse;
     for (int j = lane; j < kb; j += 32) r_lq[e * k + j] -= lse;
   }
   __syncthreads();
+  // Only now let the next wave's GEMM start: its weight stream saturates the
+  // memory system, and the partial loads above would queue behind it.
+  pdl_launch_dependents();
 
   // 2. the children become candidates, keyed by calibrated path survival
   const int n_new = rows_n * kb;
@@ -167,7 +170,14 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
       prefix += __popc(bal);
     }
     if (lane == 0) {
-      int base = prefix ? atomicAdd(f.next_count, prefix) : 0;
+      // one request: its rows start at 0 of the list the GEMM just cleared
+      int base = 0;
+      if (prefix) {
+        if (f.batch == 1)
+          *f.next_count = prefix;
+        else
+          base = atomicAdd(f.next_count, prefix);
+      }
       if (prefix && base + prefix > f.Mcap) {
         set_status(f.status, DT_EDEVICE);
         prefix = 0;
@@ -195,7 +205,7 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
         rw.key = c.key;
         f.next_rows[row] = rw;
       }
-      gather_row(f.H + (size_t)row * f.r, f.A, c.token, f.r, lane, 32);
+      if (f.H) gather_row(f.H + (size_t)row * f.r, f.A, c.token, f.r, lane, 32);
       __syncwarp();
       if (lane == 0) sorted[i].expanded = 1;
     }
@@ -245,7 +255,14 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
           if (i < n_keep) s_pos[i] = in ? (int16_t)(prefix + __popc(bal & ((1u << lane) - 1))) : -1;
           prefix += __popc(bal);
         }
-        if (lane == 0) s_cnt[3] = atomicAdd(f.mat_count, prefix);
+        if (lane == 0) {
+          if (f.batch == 1) {
+            *f.mat_count = prefix;
+            s_cnt[3] = 0;
+          } else {
+            s_cnt[3] = atomicAdd(f.mat_count, prefix);
+          }
+        }
       }
       __syncthreads();
       const int mbase = s_cnt[3];
@@ -279,7 +296,7 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
           rw.key = 0.f;
           f.mat_rows[row] = rw;
         }
-        gather_row(f.Hm + (size_t)row * f.r, f.A, token, f.r, lane, 32);
+        if (f.Hm) gather_row(f.Hm + (size_t)row * f.r, f.A, token, f.r, lane, 32);
       }
     }
   }
@@ -340,7 +357,7 @@ __global__ void build_init_kernel(FrontierArgs f, const int32_t* root_token, Row
       st.row_count = 0;
       if (lane == 0) f.out.d_n_nodes[b] = 0;
     } else {
-      gather_row(f.H + (size_t)b * f.r, f.A, root, f.r, lane, 32);
+      if (f.H) gather_row(f.H + (size_t)b * f.r, f.A, root, f.r, lane, 32);
     }
     if (lane == 0) {
       rows0[b] = rw;

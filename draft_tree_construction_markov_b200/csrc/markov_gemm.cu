@@ -77,7 +77,7 @@ struct ColMeta {
   float lse;
   int32_t out_row;
   int32_t bslot;     // row of the shared-memory bias cache (-1: not cached)
-  int32_t pad;
+  int32_t token;     // the column's token (row of A gathered as the B operand)
 };
 
 // Most distinct bias rows a CTA keeps in shared memory for its vocabulary range.
@@ -95,10 +95,12 @@ __host__ __device__ inline size_t gemm_epi_bytes(int mode, int kmax, bool stoch)
 }
 
 template <int NG>
-static size_t gemm_smem_bytes(int stages, int mode, int kmax, bool stoch, size_t bias_bytes) {
+static size_t gemm_smem_bytes(int stages, int mode, int kmax, bool stoch, size_t bias_bytes,
+                              size_t gather_bytes) {
   using S = GemmShape<NG>;
   size_t off = 1024;  // alignment slack
-  off += (size_t)stages * S::kStageBytes;
+  off += gather_bytes ? (size_t)stages * S::kABytes + gather_bytes
+                      : (size_t)stages * S::kStageBytes;
   off += (size_t)(2 * stages + 2 * S::kAccBufs + 5) * 8;  // barriers
   off += 16;                                             // tmem slot + abort flag
   off = (off + 15) & ~(size_t)15;
@@ -242,10 +244,17 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
   const int stages = a.stages;
   const int k = a.k;
 
+  // Markov columns: the B operand rows A[token] are gathered once into shared
+  // memory (resident for every stage) instead of streamed with each stage.
+  const bool gather = a.gatherA != nullptr;
+  const int sbytes = gather ? S::kABytes : S::kStageBytes;  // bytes per stage
+
   // ---- carve shared memory
   uint8_t* p = smem;
   uint8_t* stage_mem = p;
-  p += (size_t)stages * S::kStageBytes;
+  p += (size_t)stages * sbytes;
+  uint8_t* bres = p;  // gathered B rows: [KC][NT][128 B], 128-byte swizzle
+  if (gather) p += (size_t)KC * S::NT * 128;
   uint64_t* full = (uint64_t*)p;
   uint64_t* empty = full + stages;
   uint64_t* tfull = empty + stages;
@@ -309,7 +318,7 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < npre; ++i) {
       const int t = t0 + i / KC, kc = i % KC;
-      uint8_t* sa = stage_mem + (size_t)i * S::kStageBytes;
+      uint8_t* sa = stage_mem + (size_t)i * sbytes;
       mbar_expect_tx(&full[i], S::kABytes);
       if (MODE == EPI_SWIGLU) {
         // 64 gate rows, then the 64 up rows of the same features
@@ -341,7 +350,7 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
     cm.lse = 0.f;
     cm.out_row = 0;
     cm.bslot = -1;
-    cm.pad = 0;
+    cm.token = 0;
     if (row < M) {
       const Row r = a.rows[row];
       if (r.b >= 0) {
@@ -355,10 +364,35 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
           cm.c2 = (uint32_t)(r.path >> 32);
           cm.lse = r.lse;
           cm.out_row = r.aux;
+          cm.token = r.token;
+          if (gather && (r.token < 0 || r.token >= a.V)) {
+            set_status(a.status, DT_EDEVICE);
+            cm.valid = 0;
+          }
         }
       }
     }
     meta[c] = cm;
+  }
+  __syncthreads();
+  if (gather && active) {
+    // 16-byte pieces of A[token] into the swizzled K-major layout the MMA
+    // descriptors expect; columns without a node and K beyond r read as zero
+    const int npieces = KC * S::NT * 8;
+    for (int idx = threadIdx.x; idx < npieces; idx += blockDim.x) {
+      const int ch = idx & 7, c = (idx >> 3) % S::NT, kc = (idx >> 3) / S::NT;
+      const int col_k = kc * 64 + ch * 8;
+      const bool ok = meta[c].valid && col_k < a.r;
+      const uint16_t* src = ok ? a.gatherA + (size_t)meta[c].token * a.r + col_k : a.gatherA;
+      uint8_t* dst = bres + ((size_t)kc * S::NT + c) * 128 + ((ch ^ (c & 7)) << 4);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),
+                   "l"(src), "r"(ok ? 16 : 0)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    // the tensor cores read these bytes through the async proxy
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   __syncthreads();
   // The epilogues read their bias rows from shared memory: global loads
@@ -408,9 +442,13 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
       bool ok = true;
       uint32_t issued = 0, last_parity = 0;  // per stage: issued at least once, parity of last issue
       for (int i = 0; i < npre; ++i) {
-        uint8_t* sa = stage_mem + (size_t)i * S::kStageBytes;
-        mbar_arrive_expect_tx(&full[i], S::kBBytes);
-        tma_load_2d(sa + S::kABytes, &tmH, &full[i], (i % KC) * 64, ny * S::NT);
+        uint8_t* sa = stage_mem + (size_t)i * sbytes;
+        if (gather) {
+          mbar_arrive(&full[i]);
+        } else {
+          mbar_arrive_expect_tx(&full[i], S::kBBytes);
+          tma_load_2d(sa + S::kABytes, &tmH, &full[i], (i % KC) * 64, ny * S::NT);
+        }
         issued |= 1u << i;
       }
       const int n_all = active ? total : npre;
@@ -422,15 +460,15 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
           ok = false;
           break;
         }
-        uint8_t* sa = stage_mem + (size_t)stage * S::kStageBytes;
-        mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+        uint8_t* sa = stage_mem + (size_t)stage * sbytes;
+        mbar_arrive_expect_tx(&full[stage], sbytes);
         if (MODE == EPI_SWIGLU) {
           tma_load_2d(sa, &tmW, &full[stage], kc * 64, t * 64);
           tma_load_2d(sa + S::kABytes / 2, &tmW2, &full[stage], kc * 64, t * 64);
         } else {
           tma_load_2d(sa, &tmW, &full[stage], kc * 64, t * kTileV);
         }
-        tma_load_2d(sa + S::kABytes, &tmH, &full[stage], kc * 64, ny * S::NT);
+        if (!gather) tma_load_2d(sa + S::kABytes, &tmH, &full[stage], kc * 64, ny * S::NT);
         issued |= 1u << stage;
         last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
       }
@@ -464,9 +502,10 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(stage_mem + (size_t)stage * S::kStageBytes);
+          const uint32_t sa = smem_u32(stage_mem + (size_t)stage * sbytes);
           const uint64_t da = smem_desc_k_sw128(sa);
-          const uint64_t db = smem_desc_k_sw128(sa + S::kABytes);
+          const uint64_t db = smem_desc_k_sw128(
+              gather ? smem_u32(bres + (size_t)kc * S::NT * 128) : sa + S::kABytes);
           const int ks = (kc == KC - 1) ? ks_last : 4;
           for (int s = 0; s < ks; ++s)
             tc_mma_bf16(d_tmem, da + 2 * s, db + 2 * s, idesc, (kc | s) != 0 ? 1u : 0u);
@@ -834,8 +873,10 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
       for (int lst = 0; lst < (STOCH ? 2 : 1); ++lst) {
         const float* LV = lst ? ql2v : ql1v;
         const int32_t* LI = lst ? ql2i : ql1i;
-        float* OV = (lst ? a.pgv : a.plv) + pidx * k;
-        int32_t* OI = (lst ? a.pgi : a.pli) + pidx * k;
+        // list entry i of this CTA at [row][i][cta]: a merging warp reads one
+        // entry of 32 consecutive CTAs per load
+        float* OV = (lst ? a.pgv : a.plv) + (size_t)row * k * a.ncta_v + cx;
+        int32_t* OI = (lst ? a.pgi : a.pli) + (size_t)row * k * a.ncta_v + cx;
         int h0 = 0, h1 = 0, h2 = 0, h3 = 0;  // heads of the four quadrant lists
         for (int i = 0; i < k; ++i) {
           int bw = -1;
@@ -857,8 +898,8 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
           h1 += bw == 1;
           h2 += bw == 2;
           h3 += bw == 3;
-          OV[i] = bv;
-          OI[i] = bi;
+          OV[(size_t)i * a.ncta_v] = bv;
+          OI[(size_t)i * a.ncta_v] = bi;
         }
       }
     }
@@ -927,13 +968,17 @@ static cudaError_t launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmW2,
       bias_bytes = bytes;
     }
   }
+  // gathered B rows: KC x NT x 128 B, only while that stays small
+  const size_t gather_bytes = ((a.r + 63) / 64) * (size_t)SH::NT * 128;
+  if (a.gatherA && (MODE == EPI_SWIGLU || gather_bytes > 32 * 1024)) return cudaErrorInvalidValue;
+  const size_t gb = a.gatherA ? gather_bytes : 0;
   // the deepest pipeline that fits in 200 KB of shared memory, which leaves room
   // on each SM for a small kernel of the wave loop running alongside
-  int stages = 10;
-  while (stages > 2 && gemm_smem_bytes<NG>(stages, MODE, KMAX, STOCH, bias_bytes) > 200 * 1024)
+  int stages = 12;
+  while (stages > 2 && gemm_smem_bytes<NG>(stages, MODE, KMAX, STOCH, bias_bytes, gb) > 200 * 1024)
     --stages;
   a.stages = stages;
-  const size_t smem = gemm_smem_bytes<NG>(stages, MODE, KMAX, STOCH, bias_bytes);
+  const size_t smem = gemm_smem_bytes<NG>(stages, MODE, KMAX, STOCH, bias_bytes, gb);
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.ncta_v * a.n_ntiles);
@@ -949,7 +994,11 @@ int gemm_node_tile(int max_cols) { return max_cols <= 32 ? 32 : max_cols <= 64 ?
 int gemm_kmax(int k) { return k <= 4 ? 4 : 16; }
 
 // Launches one GEMM.  tmW: weight rows (box 128 rows; SwiGLU: the gate rows,
-// box 64, with tmW2 the up rows); tmH: node rows (box nt rows).
+// box 64, with tmW2 the up rows); tmH: node rows (box nt rows), unused when
+// a.gatherA is set (the rows A[token] are then gathered by the kernel).
+// Whether a launch can gather its rows.
+bool gemm_can_gather(int r, int nt) { return ((r + 63) / 64) * (size_t)nt * 128 <= 32 * 1024; }
+
 cudaError_t launch_markov_gemm(int mode, bool stoch, const CUtensorMap& tmW,
                                const CUtensorMap& tmW2, const CUtensorMap& tmH, GemmArgs a,
                                int batch, int nt, cudaStream_t s) {
