@@ -17,6 +17,8 @@ accept       greedy and recursive-residual acceptance walk (TreeSpark article,
 verify_attn  tree-masked GQA attention over prefix + root + ancestors.
 treeflash    SwiGLU AR-approximator round (TreeFlash explainer, method
              sections 1 and 2).
+variants     the baseline trees of the PCTree summary's mechanism isolation
+             (chain, marginal-ranked, Shared-Markov) and acceptance length.
 
 Every floating quantity is fp64; inputs are the exact stored values.
 """

@@ -148,7 +148,7 @@ Sampler = Callable[[tuple, np.ndarray, float, int], np.ndarray]
 
 def build_tree(L, A, Bt, root_token, k, N, temp=0.0, lam=0.0, calib=None,
                seed=0, offset=0, request=0, sampler: Optional[Sampler] = None,
-               key_mode="order_stat") -> Tree:
+               key_mode="order_stat", cond_tokens=None) -> Tree:
     """Sequential best-first construction of one request's draft tree.
 
     L: (Bk, V) block logits of this request; A, Bt: (V, r) Markov factors.
@@ -156,6 +156,12 @@ def build_tree(L, A, Bt, root_token, k, N, temp=0.0, lam=0.0, calib=None,
     the exact-enumeration tests).  ``key_mode="own_q"`` is a deliberately
     wrong variant (keys from the sampled token's own probability) that the
     tests use as a negative control; the method uses ``"order_stat"``.
+
+    ``cond_tokens`` (length Bk) replaces the parent token in the Markov term
+    for the baseline variants of the PCTree summary's mechanism-isolation
+    paragraph: every node at depth d draws its children from
+    L[d] + A[cond_tokens[d]] . B^T, or from L[d] alone where the entry is -1.
+    None (the method) conditions each node on its own token.
     """
     L = np.asarray(L)
     Bk, V = L.shape
@@ -167,8 +173,17 @@ def build_tree(L, A, Bt, root_token, k, N, temp=0.0, lam=0.0, calib=None,
     margins: list = []
     expansions: dict = {}
 
+    if cond_tokens is not None and len(cond_tokens) != Bk:
+        raise ValueError("cond_tokens needs one entry per block row")
+
+    def markov_row(depth, token):
+        if cond_tokens is None:
+            return A[token]
+        c = int(cond_tokens[depth])
+        return np.zeros(A.shape[1]) if c < 0 else A[c]
+
     def expand(row, depth, token, ranks):
-        z = node_logits(L[depth], A[token], Bt)
+        z = node_logits(L[depth], markov_row(depth, token), Bt)
         s, lse = scaled_logits(z, temp)
         order = top_k_desc(s, k)
         logq = s[order] - lse
