@@ -71,16 +71,22 @@ def accept_workspace_bytes(batch, Nmax, V) -> int:
 
 def tree_build(block_logits, markov_a, markov_b, root_token, n_budget, lam, *, k, Nmax, temp,
                out: Tree, ws, calib=None, k_req=None, philox_seed=0, philox_offset=0,
-               stream=None):
-    """dt_tree_build.  block_logits [batch,Bk,V] fp32|bf16; markov_a/markov_b [V,r] bf16."""
+               stream=None, variant="pctree"):
+    """dt_tree_build (variant "pctree") or dt_tree_build_ex with a baseline
+    variant ("chain", "marginal", "shared_markov").  block_logits
+    [batch,Bk,V] fp32|bf16; markov_a/markov_b [V,r] bf16."""
     batch, Bk, V = block_logits.shape
     r = markov_a.shape[1]
     st = out.c_struct()
-    check(_lib.lib.dt_tree_build(
-        ptr(block_logits), dtype_code(block_logits), ptr(markov_a), ptr(markov_b), r, ptr(calib),
-        ptr(root_token), ptr(n_budget), ptr(k_req), ptr(lam), batch, Bk, V, k, Nmax, float(temp),
-        philox_seed, philox_offset, ctypes.byref(st), ptr(ws), ws.numel(), stream_ptr(stream)),
-        "dt_tree_build")
+    args = (ptr(block_logits), dtype_code(block_logits), ptr(markov_a), ptr(markov_b), r,
+            ptr(calib), ptr(root_token), ptr(n_budget), ptr(k_req), ptr(lam), batch, Bk, V, k,
+            Nmax, float(temp), philox_seed, philox_offset)
+    tail = (ctypes.byref(st), ptr(ws), ws.numel(), stream_ptr(stream))
+    if variant == "pctree":
+        check(_lib.lib.dt_tree_build(*args, *tail), "dt_tree_build")
+    else:
+        check(_lib.lib.dt_tree_build_ex(*args, _lib.TREE_VARIANTS[variant], *tail),
+              "dt_tree_build_ex")
     return out
 
 

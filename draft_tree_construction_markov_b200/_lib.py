@@ -16,6 +16,7 @@ DT_OK, DT_EINVAL, DT_EUNSUPPORTED, DT_ECUDA, DT_ETIMEOUT, DT_EWORKSPACE, DT_EDEV
 STATUS_NAMES = {0: "DT_OK", 1: "DT_EINVAL", 2: "DT_EUNSUPPORTED", 3: "DT_ECUDA",
                 4: "DT_ETIMEOUT", 5: "DT_EWORKSPACE", 6: "DT_EDEVICE"}
 DT_F32, DT_BF16 = 0, 1
+TREE_VARIANTS = {"pctree": 0, "chain": 1, "marginal": 2, "shared_markov": 3}
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -43,6 +44,8 @@ _sig("dt_num_sms", _i32)
 _sig("dt_tree_build_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("dt_tree_build", _i32, _vp, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
      _i32, _i32, _i32, _i32, _i32, _f32, _u64, _u64, ctypes.POINTER(DtTree), _vp, _sz, _vp)
+_sig("dt_tree_build_ex", _i32, _vp, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
+     _i32, _i32, _i32, _i32, _i32, _f32, _u64, _u64, _i32, ctypes.POINTER(DtTree), _vp, _sz, _vp)
 _sig("dt_markov_logits_workspace_bytes", _sz, _i32, _i32, _i32)
 _sig("dt_markov_logits", _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
      _i32, _vp, _vp, _sz, _vp)

@@ -94,13 +94,15 @@ struct BuildLayout {
   int32_t* pli;
   float* pgv;
   int32_t* pgi;
+  int32_t* cond;       // [batch][Bk] per-depth Markov-row tokens of a baseline variant
+  int32_t* chain_nb;   // [batch] Shared-Markov chain: node budget min(Bk, n_budget)
+  float* chain_lam;    // [batch] Shared-Markov chain: no survival stop
   size_t bytes;
   int ncta_v, n_vtiles, nt, Mcap, Mcap_pad, Mmat, Mmat_pad;
 };
 
 static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k, int Nmax) {
   BuildLayout L;
-  (void)Bk;
   L.n_vtiles = (V + 127) / 128;
   L.ncta_v = std::min(num_sms(), L.n_vtiles);
   L.nt = gemm_node_tile(Nmax);
@@ -125,9 +127,97 @@ static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k
   L.pli = c.take<int32_t>(np * k);
   L.pgv = c.take<float>(np * k);
   L.pgi = c.take<int32_t>(np * k);
+  L.cond = c.take<int32_t>((size_t)batch * Bk);
+  L.chain_nb = c.take<int32_t>(batch);
+  L.chain_lam = c.take<float>(batch);
   L.bytes = align_up(c.off, 256);
   return L;
 }
+
+// Per-request set-up of a baseline variant (one thread per request): no
+// Markov row at any depth yet (the marginal-ranked tree keeps this), and the
+// budget of the greedy chain that the Shared-Markov tree walks first:
+// min(Bk, n_budget) nodes, no survival stop.
+__global__ void variant_prep_kernel(const int32_t* n_budget, int batch, int Bk, int Nmax,
+                                    int32_t* cond, int32_t* chain_nb, float* chain_lam) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
+    for (int d = 0; d < Bk; ++d) cond[(size_t)b * Bk + d] = -1;
+    int nb = n_budget[b];
+    nb = nb < 0 ? 0 : (nb > Nmax ? Nmax : nb);  // the build flags a budget above Nmax
+    chain_nb[b] = min(Bk, nb);
+    chain_lam[b] = 0.f;
+  }
+}
+
+// Shared-Markov conditioning from the greedy chain: depth 0 uses the root,
+// depth d >= 1 the chain's depth-d token (one thread per request).
+__global__ void chain_cond_kernel(dt_tree chain, const int32_t* root, int batch, int Bk, int Nmax,
+                                  int V, int32_t* cond) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
+    const int rt = root[b];
+    cond[(size_t)b * Bk] = (rt >= 0 && rt < V) ? rt : -1;  // a bad root is flagged by the build
+    int n = chain.d_n_nodes[b];
+    n = n < 0 ? 0 : (n > Nmax ? Nmax : n);
+    for (int i = 0; i < n; ++i) {
+      const int d = chain.d_depths[(size_t)b * Nmax + i];
+      const int t = chain.d_tokens[(size_t)b * Nmax + i];
+      if (d >= 1 && d < Bk && t >= 0 && t < V) cond[(size_t)b * Bk + d] = t;
+    }
+  }
+}
+
+
+// init + Bk waves of GEMM and frontier (+ the draft-q pass at T > 0)
+static dt_status run_waves(FrontierArgs f, GemmArgs g, const BuildLayout& L,
+                           const int32_t* d_root_token, const CUtensorMap& tmW,
+                           const CUtensorMap& tmH, const CUtensorMap& tmHm, int batch, int Bk,
+                           int Nmax, float* d_draft_q, cudaStream_t s) {
+  {
+    ProfileScope ps(DT_K_BUILD_INIT, s);
+    if (launch_build_init(f, d_root_token, L.rows[0], L.counts + 0, s) != cudaSuccess)
+      return DT_ECUDA;
+  }
+  const bool stoch = f.temp > 0.f;
+  for (int w = 0; w < Bk; ++w) {
+    const int cur = w & 1, nxt = cur ^ 1;
+    g.rows = L.rows[cur];
+    g.n_rows = L.counts + cur;
+    g.reset_count = L.counts + nxt;
+    {
+      ProfileScope ps(DT_K_MARKOV_GEMM, s);
+      if (launch_markov_gemm(EPI_EXPAND, stoch, tmW, tmW, tmH, g, batch, L.nt, s) != cudaSuccess)
+        return DT_ECUDA;
+    }
+    f.rows = L.rows[cur];
+    f.next_rows = L.rows[nxt];
+    f.next_count = L.counts + nxt;
+    {
+      ProfileScope ps(DT_K_FRONTIER, s);
+      if (launch_frontier(f, s) != cudaSuccess) return DT_ECUDA;
+    }
+  }
+  if (stoch) {
+    GemmArgs gq = g;
+    gq.rows = L.mat_rows;
+    gq.n_rows = L.counts + 2;
+    gq.reset_count = nullptr;
+    gq.Mcap = L.Mmat;
+    gq.out = d_draft_q;
+    gq.nmax1 = Nmax + 1;
+    ProfileScope ps(DT_K_DRAFT_Q, s);
+    if (launch_markov_gemm(EPI_QROWS, true, tmW, tmW, tmHm, gq, batch, L.nt, s) != cudaSuccess)
+      return DT_ECUDA;
+  }
+  return DT_OK;
+}
+
+static dt_status build_impl(const void* d_block_logits, dt_dtype ldt, const uint16_t* d_markov_a,
+                            const uint16_t* d_markov_b, int r, const float* d_calib,
+                            const int32_t* d_root_token, const int32_t* d_n_budget,
+                            const int32_t* d_k_req, const float* d_lambda, int batch, int Bk,
+                            int V, int k, int Nmax, float temp, uint64_t philox_seed,
+                            uint64_t philox_offset, int variant, const dt_tree* out, void* ws,
+                            size_t ws_bytes, cudaStream_t s);
 
 }  // namespace dt
 
@@ -156,6 +246,37 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
                         int k, int Nmax, float temp, uint64_t philox_seed,
                         uint64_t philox_offset, const dt_tree* out, void* ws, size_t ws_bytes,
                         dt_stream stream) {
+  return build_impl(d_block_logits, ldt, d_markov_a, d_markov_b, r, d_calib, d_root_token,
+                    d_n_budget, d_k_req, d_lambda, batch, Bk, V, k, Nmax, temp, philox_seed,
+                    philox_offset, DT_TREE_PCTREE, out, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+dt_status dt_tree_build_ex(const void* d_block_logits, dt_dtype ldt, const uint16_t* d_markov_a,
+                           const uint16_t* d_markov_b, int r, const float* d_calib,
+                           const int32_t* d_root_token, const int32_t* d_n_budget,
+                           const int32_t* d_k_req, const float* d_lambda, int batch, int Bk,
+                           int V, int k, int Nmax, float temp, uint64_t philox_seed,
+                           uint64_t philox_offset, dt_tree_variant variant, const dt_tree* out,
+                           void* ws, size_t ws_bytes, dt_stream stream) {
+  if (variant != DT_TREE_PCTREE && variant != DT_TREE_CHAIN && variant != DT_TREE_MARGINAL &&
+      variant != DT_TREE_SHARED_MARKOV)
+    return DT_EINVAL;
+  return build_impl(d_block_logits, ldt, d_markov_a, d_markov_b, r, d_calib, d_root_token,
+                    d_n_budget, d_k_req, d_lambda, batch, Bk, V, k, Nmax, temp, philox_seed,
+                    philox_offset, variant, out, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+}  // extern "C"
+
+namespace dt {
+
+static dt_status build_impl(const void* d_block_logits, dt_dtype ldt, const uint16_t* d_markov_a,
+                            const uint16_t* d_markov_b, int r, const float* d_calib,
+                            const int32_t* d_root_token, const int32_t* d_n_budget,
+                            const int32_t* d_k_req, const float* d_lambda, int batch, int Bk,
+                            int V, int k, int Nmax, float temp, uint64_t philox_seed,
+                            uint64_t philox_offset, int variant, const dt_tree* out, void* ws,
+                            size_t ws_bytes, cudaStream_t s) {
   if (!d_block_logits || !d_markov_a || !d_markov_b || !d_root_token || !d_n_budget ||
       !d_lambda || !out)
     return DT_EINVAL;
@@ -172,7 +293,6 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   BuildLayout L = build_layout(nullptr, batch, Bk, V, r, k, Nmax);
   if (!ws || ws_bytes < L.bytes) return DT_EWORKSPACE;
   L = build_layout(ws, batch, Bk, V, r, k, Nmax);
-  cudaStream_t s = (cudaStream_t)stream;
 
   CUtensorMap tmW, tmH, tmHm;
   if (!make_tmap_bf16_kmajor(&tmW, d_markov_b, r, V, 128) ||
@@ -238,44 +358,42 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt, const uint16_t
   g.nmax1 = Nmax + 1;
   g.status = L.status;
 
-
-  {
-    ProfileScope ps(DT_K_BUILD_INIT, s);
-    if (launch_build_init(f, d_root_token, L.rows[0], L.counts + 0, s) != cudaSuccess)
-      return DT_ECUDA;
+  if (variant == DT_TREE_CHAIN) {
+    // the method with one child per node (k = 1 everywhere)
+    f.k = g.k = 1;
+    f.k_req = nullptr;
   }
-  const bool stoch = temp > 0.f;
-  for (int w = 0; w < Bk; ++w) {
-    const int cur = w & 1, nxt = cur ^ 1;
-    g.rows = L.rows[cur];
-    g.n_rows = L.counts + cur;
-    g.reset_count = L.counts + nxt;
-    {
-      ProfileScope ps(DT_K_MARKOV_GEMM, s);
-      if (launch_markov_gemm(EPI_EXPAND, stoch, tmW, tmW, tmH, g, batch, L.nt, s) != cudaSuccess)
-        return DT_ECUDA;
-    }
-    f.rows = L.rows[cur];
-    f.next_rows = L.rows[nxt];
-    f.next_count = L.counts + nxt;
-    {
-      ProfileScope ps(DT_K_FRONTIER, s);
-      if (launch_frontier(f, s) != cudaSuccess) return DT_ECUDA;
-    }
+  if (variant == DT_TREE_MARGINAL || variant == DT_TREE_SHARED_MARKOV) {
+    variant_prep_kernel<<<(batch + 127) / 128, 128, 0, s>>>(d_n_budget, batch, Bk, Nmax, L.cond,
+                                                           L.chain_nb, L.chain_lam);
+    if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
   }
-  if (stoch) {
-    GemmArgs gq = g;
-    gq.rows = L.mat_rows;
-    gq.n_rows = L.counts + 2;
-    gq.reset_count = nullptr;
-    gq.Mcap = L.Mmat;
-    gq.out = out->d_draft_q;
-    ProfileScope ps(DT_K_DRAFT_Q, s);
-    if (launch_markov_gemm(EPI_QROWS, true, tmW, tmW, tmHm, gq, batch, L.nt, s) != cudaSuccess)
-      return DT_ECUDA;
+  if (variant == DT_TREE_MARGINAL) f.cond = L.cond;
+  if (variant == DT_TREE_SHARED_MARKOV) {
+    // walk the greedy chain first (into the caller's tree arrays, which the
+    // tree build then overwrites), then condition depth d on its token
+    FrontierArgs fc = f;
+    GemmArgs gc = g;
+    fc.n_budget = L.chain_nb;
+    fc.k = gc.k = 1;
+    fc.k_req = nullptr;
+    fc.lambda = L.chain_lam;
+    fc.temp = 0.f;
+    gc.temp = 0.f;
+    const dt_status st = run_waves(fc, gc, L, d_root_token, tmW, tmH, tmHm, batch, Bk, Nmax,
+                                   nullptr, s);
+    if (st != DT_OK) return st;
+    chain_cond_kernel<<<(batch + 127) / 128, 128, 0, s>>>(*out, d_root_token, batch, Bk, Nmax, V,
+                                                         L.cond);
+    if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+    f.cond = L.cond;
   }
-  return DT_OK;
+  return run_waves(f, g, L, d_root_token, tmW, tmH, tmHm, batch, Bk, Nmax, out->d_draft_q, s);
 }
+
+}  // namespace dt
+
+extern "C" {
 
 // ---------------------------------------------------------------- z rows --
 namespace {

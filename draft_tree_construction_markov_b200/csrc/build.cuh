@@ -8,7 +8,7 @@ namespace dt {
 struct __align__(32) Row {
   int32_t b;      // request (-1 = padding column)
   int32_t depth;  // depth of the node; its children use block-logit row `depth`
-  int32_t token;  // token of the node (selects the Markov-head row A[token])
+  int32_t token;  // Markov-head row A[token] of the node's children (-1: no Markov term)
   int32_t aux;    // expand: node serial (-1 = root); q/z rows: output row
   uint64_t path;  // path id (Philox counter words 1-2)
   float lse;      // q rows: log-sum-exp of the node's scaled logits
@@ -92,6 +92,7 @@ struct FrontierArgs {
   uint16_t* H;           // gathered Markov rows of the next wave [Mcap][r] (NULL: the GEMM gathers)
   uint16_t* Hm;          // gathered Markov rows of mat_rows (NULL: the GEMM gathers)
   const uint16_t* A;     // [V][r]
+  const int32_t* cond;   // [batch][Bk] Markov-row token per depth (-1: none); NULL: own token
   ReqState* req;
   Cand* lists;           // [batch][Nmax]
   const float2* pstats;  // per-CTA partials of the wave GEMM (see GemmArgs)

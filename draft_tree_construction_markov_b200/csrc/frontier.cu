@@ -26,11 +26,23 @@ __device__ __forceinline__ uint64_t sort_key(const Cand& c, int idx) {
   return ((uint64_t)hi << 32) | lo;
 }
 
+// Row A[token] of the Markov head (zeros for token -1) into H.
 __device__ __forceinline__ void gather_row(uint16_t* dst, const uint16_t* A, int token, int r,
                                            int lane, int nlanes) {
-  const uint4* s = (const uint4*)(A + (size_t)token * r);
   uint4* d = (uint4*)dst;
+  if (token < 0) {
+    for (int i = lane; i < r / 8; i += nlanes) d[i] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  const uint4* s = (const uint4*)(A + (size_t)token * r);
   for (int i = lane; i < r / 8; i += nlanes) d[i] = s[i];
+}
+
+// Token whose Markov row conditions the children of a node of request b at
+// depth d: the node's own token (the method), or the per-depth token of a
+// baseline variant (-1 = block logits alone).
+__device__ __forceinline__ int markov_token(const FrontierArgs& f, int b, int depth, int token) {
+  return f.cond ? f.cond[(size_t)b * f.Bk + depth] : token;
 }
 
 template <int KMAX>
@@ -198,14 +210,15 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
         Row rw;
         rw.b = b;
         rw.depth = c.depth;
-        rw.token = c.token;
+        rw.token = markov_token(f, b, c.depth, c.token);
         rw.aux = c.serial;
         rw.path = c.path;
         rw.lse = 0.f;
         rw.key = c.key;
         f.next_rows[row] = rw;
       }
-      if (f.H) gather_row(f.H + (size_t)row * f.r, f.A, c.token, f.r, lane, 32);
+      if (f.H) gather_row(f.H + (size_t)row * f.r, f.A, markov_token(f, b, c.depth, c.token), f.r,
+                          lane, 32);
       __syncwarp();
       if (lane == 0) sorted[i].expanded = 1;
     }
@@ -284,6 +297,7 @@ __global__ void __launch_bounds__(kFrontierThreads) frontier_kernel(FrontierArgs
           aux = i + 1;
           lse = c.lse;
         }
+        token = markov_token(f, b, depth, token);
         const int row = mbase + pos;
         if (lane == 0) {
           Row rw;
@@ -346,7 +360,7 @@ __global__ void build_init_kernel(FrontierArgs f, const int32_t* root_token, Row
     Row rw;
     rw.b = b;
     rw.depth = 0;
-    rw.token = root;
+    rw.token = markov_token(f, b, 0, root);
     rw.aux = -1;
     rw.path = 0;
     rw.lse = 0.f;
@@ -357,7 +371,7 @@ __global__ void build_init_kernel(FrontierArgs f, const int32_t* root_token, Row
       st.row_count = 0;
       if (lane == 0) f.out.d_n_nodes[b] = 0;
     } else {
-      if (f.H) gather_row(f.H + (size_t)b * f.r, f.A, root, f.r, lane, 32);
+      if (f.H) gather_row(f.H + (size_t)b * f.r, f.A, rw.token, f.r, lane, 32);
     }
     if (lane == 0) {
       rows0[b] = rw;

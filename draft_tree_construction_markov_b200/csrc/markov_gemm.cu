@@ -365,7 +365,8 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
           cm.lse = r.lse;
           cm.out_row = r.aux;
           cm.token = r.token;
-          if (gather && (r.token < 0 || r.token >= a.V)) {
+          // token -1: no Markov term (zero row); anything else must index A
+          if (gather && (r.token < -1 || r.token >= a.V)) {
             set_status(a.status, DT_EDEVICE);
             cm.valid = 0;
           }
@@ -377,12 +378,13 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
   __syncthreads();
   if (gather && active) {
     // 16-byte pieces of A[token] into the swizzled K-major layout the MMA
-    // descriptors expect; columns without a node and K beyond r read as zero
+    // descriptors expect; columns without a node, token -1 (no Markov term)
+    // and K beyond r read as zero
     const int npieces = KC * S::NT * 8;
     for (int idx = threadIdx.x; idx < npieces; idx += blockDim.x) {
       const int ch = idx & 7, c = (idx >> 3) % S::NT, kc = (idx >> 3) / S::NT;
       const int col_k = kc * 64 + ch * 8;
-      const bool ok = meta[c].valid && col_k < a.r;
+      const bool ok = meta[c].valid && meta[c].token >= 0 && col_k < a.r;
       const uint16_t* src = ok ? a.gatherA + (size_t)meta[c].token * a.r + col_k : a.gatherA;
       uint8_t* dst = bres + ((size_t)kc * S::NT + c) * 128 + ((ch ^ (c & 7)) << 4);
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),

@@ -4,6 +4,8 @@
  * One decode round of parent-conditioned draft-tree speculative decoding:
  *   dt_tree_build       expand a budget-N draft tree best-first from one block
  *                       of drafter logits and a low-rank Markov head
+ *   dt_tree_build_ex    the same, or one of the baseline trees it is compared
+ *                       with (chain, marginal-ranked, Shared-Markov)
  *   dt_tree_verify_attn tree-masked grouped-query attention over prefix + tree
  *   dt_tree_accept      lossless acceptance walk (greedy or recursive residual)
  *
@@ -117,6 +119,43 @@ dt_status dt_tree_build(const void* d_block_logits, dt_dtype ldt,
                         uint64_t philox_seed, uint64_t philox_offset,
                         const dt_tree* out, void* ws, size_t ws_bytes,
                         dt_stream stream);
+
+/* ----------------------------------------------------- baseline variants --
+ * The trees that the PCTree summary's mechanism isolation compares with the
+ * parent-conditioned tree (Shared-Markov paragraph; mechanism-isolation
+ * paragraph and results table: acceptance length chain < Shared-Markov <
+ * PCTree on the same drafter weights).  Every variant runs the same kernels
+ * as dt_tree_build and differs only in which token's Markov row conditions
+ * the children of a depth-d node:
+ *   DT_TREE_PCTREE         the node's own token (exactly dt_tree_build)
+ *   DT_TREE_CHAIN          the node's own token with k = 1 for every request
+ *                          (d_k_req ignored): the drafter's chain
+ *   DT_TREE_MARGINAL       none: z_u = L[b][d] (block logits alone)
+ *   DT_TREE_SHARED_MARKOV  c_d: the greedy (T = 0, k = 1, lambda = 0) chain of
+ *                          min(Bk, n_budget[b]) nodes is built first, c_0 =
+ *                          the root and c_d its depth-d token; every node of
+ *                          depth d then draws its children from
+ *                          L[b][d] + A[c_d] . Bm, at the call's temperature.
+ * The chain walk of DT_TREE_SHARED_MARKOV writes the caller's tree arrays
+ * before the tree overwrites them.  Arguments, limits, workspace size
+ * (dt_tree_build_workspace_bytes) and errors are those of dt_tree_build;
+ * an unknown variant returns DT_EINVAL. */
+typedef enum {
+  DT_TREE_PCTREE = 0,
+  DT_TREE_CHAIN = 1,
+  DT_TREE_MARGINAL = 2,
+  DT_TREE_SHARED_MARKOV = 3
+} dt_tree_variant;
+
+dt_status dt_tree_build_ex(const void* d_block_logits, dt_dtype ldt,
+                           const uint16_t* d_markov_a, const uint16_t* d_markov_b,
+                           int r, const float* d_calib,
+                           const int32_t* d_root_token, const int32_t* d_n_budget,
+                           const int32_t* d_k_req, const float* d_lambda,
+                           int batch, int Bk, int V, int k, int Nmax, float temp,
+                           uint64_t philox_seed, uint64_t philox_offset,
+                           dt_tree_variant variant, const dt_tree* out, void* ws,
+                           size_t ws_bytes, dt_stream stream);
 
 /* Diagnostic: z rows for given (request, depth, token) triples, fp32
  * [n_rows][V] (d_z), through the same tensor-core GEMM the build uses. */
