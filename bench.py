@@ -39,6 +39,10 @@ DESCS = {
                  "T=0.6 stochastic (Philox), verify 32q/8kv d=128 prefix 4096, batch 1"),
     "load_adaptive": ("load-adaptive batch: 64 requests, B=7, V=151936, per-request budget from "
                       "{chain, 8, 16, 32}, lambda 0.01, T=1.0, lognormal prefixes 512..8192"),
+    "acceptance_study": ("baseline-tree acceptance study: 64 requests, V=151936, block B=16, "
+                         "N=32, Markov rank 256 (sigma 0.35), greedy; variants chain, "
+                         "marginal-ranked, Shared-Markov, PCTree k=2/4/8; verify 32q/8kv d=128 "
+                         "prefix 1024; synthetic first-order target"),
     "treeflash": ("TreeFlash tree build: SwiGLU AR-approximator d=2560, d_ff=2560, bf16 LM head "
                   "2560x151936, M=4, depth 16 (61 evaluations per request), budget B=16, "
                   "batch 16, T=0"),
@@ -54,7 +58,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--copies", type=int, default=4)
     p.add_argument("--no-oracle", action="store_true", help="skip the cpu_baseline leg")
-    p.add_argument("--workload", default=WORKLOAD, choices=["qwen3_4b", "qwen3_8b", "load_adaptive", "treeflash"])
+    p.add_argument("--workload", default=WORKLOAD, choices=["qwen3_4b", "qwen3_8b", "load_adaptive", "treeflash", "acceptance_study"])
     return p.parse_args()
 
 
@@ -590,6 +594,208 @@ def run_treeflash(args):
     print(json.dumps(out))
 
 
+def count_launches(dt, stream, fn):
+    """Library kernels one call of ``fn`` launches, through the event hook."""
+    import ctypes
+    import torch
+    cap = 512
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap)]
+    for e in evs:
+        e.record(stream)   # materialise the handles before reading them
+    torch.cuda.synchronize()
+    ev_arr = (ctypes.c_void_p * (2 * cap))(*[e.cuda_event for e in evs])
+    kinds = (ctypes.c_int32 * cap)()
+    count = ctypes.c_int32(0)
+    dt._lib.lib.dt_set_profile_events(ev_arr, kinds, cap, ctypes.byref(count))
+    with torch.cuda.stream(stream):
+        fn()
+    torch.cuda.synchronize()
+    dt._lib.lib.dt_set_profile_events(None, None, 0, None)
+    return int(count.value)
+
+
+STUDY = [("chain", 4), ("marginal", 4), ("shared_markov", 4), ("pctree", 4), ("pctree", 2),
+         ("pctree", 8)]
+
+
+def run_study(args):
+    """Accepted tokens per round of the baseline trees (one GPU).
+
+    For every (variant, k) of STUDY: build the 64 requests' trees, score them
+    with the synthetic first-order target, walk them (greedy) and time the
+    whole round (build + verify + accept) from a CUDA graph.  The headline is
+    PCTree's accepted tokens per second of these three calls; the per-variant
+    acceptance lengths are the study."""
+    import torch
+    import draft_tree_construction_markov_b200 as dt
+    from gen import attention_inputs, make_workload, target_rows
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    bf = torch.bfloat16
+    w = make_workload("acceptance_study", seed=rank)
+    V, Bk, N, r, B = w.V, w.Bk, w.Nmax, w.r, w.batch
+    kmax = max(k for _, k in STUDY)
+    P = int(w.prefix_len.max())
+    att = [attention_inputs(w, N + 1, b) for b in range(B)]
+    cu = lambda a, tt=bf: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(tt)
+    d = dict(L=cu(w.L), A=cu(w.A), Bt=cu(w.Bt), root=torch.from_numpy(w.root).to(dev),
+             nb=torch.from_numpy(w.n_budget).to(dev), lam=torch.from_numpy(w.lam).to(dev),
+             q=cu(np.stack([a_[0] for a_ in att])), kp=cu(np.concatenate([a_[1] for a_ in att])),
+             vp=cu(np.concatenate([a_[2] for a_ in att])), kt=cu(np.stack([a_[3] for a_ in att])),
+             vt=cu(np.stack([a_[4] for a_ in att])))
+    del att
+    pstart = np.concatenate([[0], np.cumsum(w.prefix_len)[:-1]]).astype(np.int64)
+    d["pstart"] = torch.from_numpy(pstart).to(dev)
+    d["plen"] = torch.from_numpy(w.prefix_len).to(dev)
+    tree = dt.Tree.empty(B, N, V, stochastic=False, device=dev)
+    ws_b = dt.workspace(dt.build_workspace_bytes(B, Bk, V, r, kmax, N), dev)
+    ws_v = dt.workspace(dt.verify_workspace_bytes(B, N, w.Hq, w.Hkv, w.d, P), dev)
+    ws_a = dt.workspace(dt.accept_workspace_bytes(B, N, V), dev)
+    attn_out = torch.empty(B, N + 1, w.Hq, w.d, dtype=bf, device=dev)
+    acc = torch.empty(B, Bk, dtype=torch.int32, device=dev)
+    nacc = torch.empty(B, dtype=torch.int32, device=dev)
+    bonus = torch.empty(B, dtype=torch.int32, device=dev)
+    tgt = torch.empty(B, N + 1, V, dtype=bf, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def round_(variant, k):
+        dt.tree_build(d["L"], d["A"], d["Bt"], d["root"], d["nb"], d["lam"], k=k, Nmax=N,
+                      temp=0.0, out=tree, ws=ws_b, variant=variant)
+        dt.tree_verify_attn(d["q"], d["kp"], d["vp"], d["pstart"], d["plen"], P, d["kt"],
+                            d["vt"], tree.anc, tree.n_nodes, 1.0 / math.sqrt(w.d), attn_out, ws_v)
+        dt.tree_accept(tgt, tree, Bk, 0.0, acc, nacc, bonus, ws_a)
+
+    res, host_trees = {}, {}
+    clocks = ClockSampler(local)
+    clocks.start()
+    for variant, k in STUDY:
+        name = variant if k == 4 else f"{variant}_k{k}"
+        with torch.cuda.stream(stream):
+            dt.tree_build(d["L"], d["A"], d["Bt"], d["root"], d["nb"], d["lam"], k=k, Nmax=N,
+                          temp=0.0, out=tree, ws=ws_b, variant=variant)
+        torch.cuda.synchronize()
+        assert dt.read_status(ws_b) == 0
+        n_nodes = tree.n_nodes.cpu().numpy()
+        toks, deps = tree.tokens.cpu().numpy(), tree.depths.cpu().numpy()
+        host_trees[name] = (n_nodes, toks, deps)
+        # the synthetic target scores this variant's trees (rows past a tree's
+        # last node are never read)
+        for b in range(B):
+            n = int(n_nodes[b])
+            rows = target_rows(w, b, np.concatenate([[0], deps[b, :n]]),
+                               np.concatenate([w.root[b:b + 1], toks[b, :n]]))
+            tgt[b, : n + 1].copy_(torch.from_numpy(rows))
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3)):
+                round_(variant, k)
+        torch.cuda.synchronize()
+        for wsx in (ws_b, ws_v, ws_a):
+            assert dt.read_status(wsx) == 0
+        tau = nacc.cpu().numpy() + 1
+        n_launch = count_launches(dt, stream, lambda: round_(variant, k))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            round_(variant, k)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                g.replay()
+            e0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        assert np.array_equal(nacc.cpu().numpy() + 1, tau)   # replays reproduce the walk
+        res[name] = {"accept_len": round(float(tau.mean()), 4),
+                     "accept_len_sem": round(float(tau.std(ddof=1) / math.sqrt(B)), 4),
+                     "tree_nodes_mean": round(float(n_nodes.mean()), 2),
+                     "ms_per_round": round(ms, 4),
+                     "request_rounds_per_s": round(B / (ms / 1e3), 1),
+                     "accepted_tokens_per_s": round(float(tau.sum()) / (ms / 1e3), 1),
+                     "launches_per_round": n_launch, "tau": tau}
+        del g
+    clk = clocks.stop()
+
+    # end to end through the Python API for PCTree: block logits, tree rows
+    # of q/k/v and the target rows from pinned host memory every round, the
+    # accept results back
+    h_in = {nm: d[nm].cpu().pin_memory() for nm in ("L", "q", "kt", "vt")}
+    h_in["tgt"] = tgt.cpu().pin_memory()
+    dst = dict(d, tgt=tgt)
+    h_out = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in (acc, nacc, bonus)]
+    ke = 5
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            for nm, hx in h_in.items():
+                dst[nm].copy_(hx, non_blocking=True)
+            round_("pctree", 4)
+            for hx, x in zip(h_out, (acc, nacc, bonus)):
+                hx.copy_(x, non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize()
+        e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e3.record(stream)
+    torch.cuda.synchronize()
+    ms_e = e2.elapsed_time(e3) / ke
+    tau_e = h_out[1].numpy() + 1
+    e2e = {"value": round(float(tau_e.sum()) / (ms_e / 1e3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in h_in.values())),
+           "d2h_bytes_per_step": int(sum(x.numel() * x.element_size() for x in h_out)),
+           "steps": ke, "path": "python API (eager launches) + pinned H2D/D2H copies"}
+    base = res["chain"]["tau"]
+    for name, v in res.items():
+        diff = v["tau"] - base
+        v["paired_gain_vs_chain"] = round(float(diff.mean()), 4)
+        v["paired_gain_sem"] = round(float(diff.std(ddof=1) / math.sqrt(B)), 4)
+    head = res["pctree"]
+    out = {
+        "metric": "accepted tokens/s of one draft-tree round (build+verify+accept), PCTree, "
+                  "acceptance-study config; per-variant acceptance lengths in 'variants'",
+        "value": head["accepted_tokens_per_s"], "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_round"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": DESCS["acceptance_study"],
+                   "l2": "Markov factors 156 MB + target rows 642 MB > 126 MB L2 per round",
+                   "round": "CUDA graph per variant"},
+        "variants": {nm: {kk: vv for kk, vv in v.items() if kk != "tau"} for nm, v in res.items()},
+        "gpu_launches": int(sum(v["launches_per_round"] * (args.steps + args.warmup)
+                                for v in res.values())),
+        "e2e": e2e, "clocks": clk,
+    }
+    if not args.no_oracle:
+        # the oracle on a bounded sample: two requests, every k = 4 variant,
+        # on the same target rows; its acceptance lengths must agree
+        from oracle import variants as ov
+        t0, agree, n_t, tok_sum = time.time(), True, 0, 0
+        A64, B64 = w.A.astype(np.float64), w.Bt.astype(np.float64)
+        for b in range(2):
+            for variant, k in STUDY[:4]:
+                o = ov.variant_tree(variant, w.L[b].astype(np.float64), A64, B64, int(w.root[b]),
+                                    k, N)
+                rows = target_rows(w, b, np.concatenate([[0], o.depths]),
+                                   np.concatenate([w.root[b:b + 1], o.tokens])).astype(np.float64)
+                tau_o = ov.acceptance_length(o, rows)
+                n_nodes, toks, _ = host_trees[variant]
+                agree &= (int(n_nodes[b]) == o.n and np.array_equal(toks[b, :o.n], o.tokens)
+                          and tau_o == int(res[variant]["tau"][b]))
+                n_t += 1
+                tok_sum += tau_o
+        el = time.time() - t0
+        out["cpu_baseline"] = {"value": round(tok_sum / el, 4), "unit": "tokens/s",
+                               "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"{n_t} trees (2 requests x 4 variants) built, scored and "
+                                         f"walked in {el:.1f} s (numpy fp64)"}
+        out["oracle_agrees"] = bool(agree)
+    print(json.dumps(out))
+
+
 def run_reference(args):
     """The oracle as the reference arm: each step is one CPU round of the workload."""
     rank, world, local = dist_env()
@@ -635,5 +841,7 @@ if __name__ == "__main__":
         run_reference(a)
     elif a.workload == "treeflash":
         run_treeflash(a)
+    elif a.workload == "acceptance_study":
+        run_study(a)
     else:
         run_ours(a)

@@ -357,6 +357,9 @@ static dt_status build_impl(const void* d_block_logits, dt_dtype ldt, const uint
   g.pgi = L.pgi;
   g.nmax1 = Nmax + 1;
   g.status = L.status;
+  // a wave's column count is only known on the device: one CTA per weight
+  // range loops over the node tiles that have columns
+  g.n_nslots = 1;
 
   if (variant == DT_TREE_CHAIN) {
     // the method with one child per node (k = 1 everywhere)
@@ -364,6 +367,7 @@ static dt_status build_impl(const void* d_block_logits, dt_dtype ldt, const uint
     f.k_req = nullptr;
   }
   if (variant == DT_TREE_MARGINAL || variant == DT_TREE_SHARED_MARKOV) {
+    ProfileScope ps(DT_K_OTHER, s);
     variant_prep_kernel<<<(batch + 127) / 128, 128, 0, s>>>(d_n_budget, batch, Bk, Nmax, L.cond,
                                                            L.chain_nb, L.chain_lam);
     if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
@@ -383,9 +387,12 @@ static dt_status build_impl(const void* d_block_logits, dt_dtype ldt, const uint
     const dt_status st = run_waves(fc, gc, L, d_root_token, tmW, tmH, tmHm, batch, Bk, Nmax,
                                    nullptr, s);
     if (st != DT_OK) return st;
-    chain_cond_kernel<<<(batch + 127) / 128, 128, 0, s>>>(*out, d_root_token, batch, Bk, Nmax, V,
-                                                         L.cond);
-    if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+    {
+      ProfileScope ps(DT_K_OTHER, s);
+      chain_cond_kernel<<<(batch + 127) / 128, 128, 0, s>>>(*out, d_root_token, batch, Bk, Nmax,
+                                                           V, L.cond);
+      if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+    }
     f.cond = L.cond;
   }
   return run_waves(f, g, L, d_root_token, tmW, tmH, tmHm, batch, Bk, Nmax, out->d_draft_q, s);

@@ -58,6 +58,8 @@ struct GemmArgs {
   int n_vtiles;          // weight tiles (128 rows; SwiGLU: 64 features)
   int ncta_v;            // weight ranges (= partials per node)
   int n_ntiles;          // node tiles for Mcap columns (set by the launcher)
+  int n_nslots;          // node-tile slots per weight range (0: one per tile); a CTA
+                         // loops over tiles slot, slot + n_nslots, ...
   int bias_span;         // bias cache row length (set by the launcher; 0 = no cache)
   int bias_rows;         // bias cache capacity in rows (set by the launcher)
   const uint16_t* gatherA;  // [V][r]: gather B rows A[token] in the kernel (NULL: TMA from H)

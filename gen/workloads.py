@@ -51,6 +51,14 @@ CONFIGS = {
                      logit_dtype="bf16", L_scale=3.0, plant=("margin", 8.0, 2.0),
                      target_sigma=1.2, P=4096, Hq=32, Hkv=8, d=128,
                      attn_dtype="bf16", batch=1, temp=0.6, lam=0.0),
+    # Acceptance study of the baseline trees: the Qwen3-8B-shaped block
+    # (B=16, k=4, N=32, greedy) with a stronger Markov term (sigma 0.35, so
+    # the next token depends on the parent more than in the rounds above),
+    # 64 requests, 1024-token prefixes.
+    "acceptance_study": dict(V=151936, Bk=16, k=4, N=32, r=256, sigma_ab=0.35,
+                             logit_dtype="bf16", L_scale=3.0, plant=("margin", 8.0, 2.0),
+                             target_sigma=1.0, P=1024, Hq=32, Hkv=8, d=128,
+                             attn_dtype="bf16", batch=64, temp=0.0, lam=0.0),
     # Load-adaptive batch: 64 requests, lognormal prefixes clipped to
     # [512, 8192], per-request budget from {chain, 8, 16, 32}, lambda 0.01, T=1.
     "load_adaptive": dict(V=151936, Bk=7, k=4, N=32, r=256, sigma_ab=0.25,

@@ -36,9 +36,14 @@ def run_variant(w, variant, temp, seed=None):
     return tree
 
 
+_F64 = {}
+
+
 def oracle_variant(w, variant, b, temp, seed=None):
+    if _F64.get("w") is not w:   # fp64 copies of the Markov factors, once per workload
+        _F64.update(w=w, A=w.A.astype(np.float64), Bt=w.Bt.astype(np.float64))
     return variants.variant_tree(
-        variant, w.L[b], w.A, w.Bt, int(w.root[b]), int(w.k_req[b]), int(w.n_budget[b]),
+        variant, w.L[b], _F64["A"], _F64["Bt"], int(w.root[b]), int(w.k_req[b]), int(w.n_budget[b]),
         temp=temp, lam=float(w.lam[b]), calib=w.calib,
         seed=w.philox_seed if seed is None else seed, request=b)
 
