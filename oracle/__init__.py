@@ -19,6 +19,8 @@ treeflash    SwiGLU AR-approximator round (TreeFlash explainer, method
              sections 1 and 2).
 variants     the baseline trees of the PCTree summary's mechanism isolation
              (chain, marginal-ranked, Shared-Markov) and acceptance length.
+load_policy  survival-ordered allocation of a round's verification capacity
+             over a batch (TreeSpark article, load-adaptive serving policy).
 
 Every floating quantity is fp64; inputs are the exact stored values.
 """
