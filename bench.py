@@ -43,6 +43,10 @@ DESCS = {
                          "N=32, Markov rank 256 (sigma 0.35), greedy; variants chain, "
                          "marginal-ranked, Shared-Markov, PCTree k=2/4/8; verify 32q/8kv d=128 "
                          "prefix 1024; synthetic first-order target"),
+    "load_policy": ("load sweep of the load-adaptive tree size: 1..64 requests, V=151936, "
+                    "block B=16, k=4, N=32, Markov rank 256 (sigma 0.35), greedy, lognormal "
+                    "prefixes 512..8192; trees cut to 256 verification units per round, a node "
+                    "costing 1 + prefix // 2048; synthetic first-order target"),
     "treeflash": ("TreeFlash tree build: SwiGLU AR-approximator d=2560, d_ff=2560, bf16 LM head "
                   "2560x151936, M=4, depth 16 (61 evaluations per request), budget B=16, "
                   "batch 16, T=0"),
@@ -58,7 +62,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--copies", type=int, default=4)
     p.add_argument("--no-oracle", action="store_true", help="skip the cpu_baseline leg")
-    p.add_argument("--workload", default=WORKLOAD, choices=["qwen3_4b", "qwen3_8b", "load_adaptive", "treeflash", "acceptance_study"])
+    p.add_argument("--workload", default=WORKLOAD, choices=["qwen3_4b", "qwen3_8b", "load_adaptive", "treeflash", "acceptance_study", "load_policy"])
     return p.parse_args()
 
 
@@ -594,6 +598,25 @@ def run_treeflash(args):
     print(json.dumps(out))
 
 
+def batch_inputs(w, dev):
+    """Device copies of a multi-request workload: block logits, Markov
+    factors, request parameters, and one attention layer's q/k/v rows."""
+    import torch
+    from gen import attention_inputs
+    bf = torch.bfloat16
+    att = [attention_inputs(w, w.Nmax + 1, b) for b in range(w.batch)]
+    cu = lambda a, tt=bf: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(tt)
+    d = dict(L=cu(w.L), A=cu(w.A), Bt=cu(w.Bt), root=torch.from_numpy(w.root).to(dev),
+             nb=torch.from_numpy(w.n_budget).to(dev), lam=torch.from_numpy(w.lam).to(dev),
+             q=cu(np.stack([a_[0] for a_ in att])), kp=cu(np.concatenate([a_[1] for a_ in att])),
+             vp=cu(np.concatenate([a_[2] for a_ in att])), kt=cu(np.stack([a_[3] for a_ in att])),
+             vt=cu(np.stack([a_[4] for a_ in att])))
+    pstart = np.concatenate([[0], np.cumsum(w.prefix_len)[:-1]]).astype(np.int64)
+    d["pstart"] = torch.from_numpy(pstart).to(dev)
+    d["plen"] = torch.from_numpy(w.prefix_len).to(dev)
+    return d
+
+
 def count_launches(dt, stream, fn):
     """Library kernels one call of ``fn`` launches, through the event hook."""
     import ctypes
@@ -628,7 +651,7 @@ def run_study(args):
     acceptance lengths are the study."""
     import torch
     import draft_tree_construction_markov_b200 as dt
-    from gen import attention_inputs, make_workload, target_rows
+    from gen import make_workload, target_rows
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -638,17 +661,7 @@ def run_study(args):
     V, Bk, N, r, B = w.V, w.Bk, w.Nmax, w.r, w.batch
     kmax = max(k for _, k in STUDY)
     P = int(w.prefix_len.max())
-    att = [attention_inputs(w, N + 1, b) for b in range(B)]
-    cu = lambda a, tt=bf: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(tt)
-    d = dict(L=cu(w.L), A=cu(w.A), Bt=cu(w.Bt), root=torch.from_numpy(w.root).to(dev),
-             nb=torch.from_numpy(w.n_budget).to(dev), lam=torch.from_numpy(w.lam).to(dev),
-             q=cu(np.stack([a_[0] for a_ in att])), kp=cu(np.concatenate([a_[1] for a_ in att])),
-             vp=cu(np.concatenate([a_[2] for a_ in att])), kt=cu(np.stack([a_[3] for a_ in att])),
-             vt=cu(np.stack([a_[4] for a_ in att])))
-    del att
-    pstart = np.concatenate([[0], np.cumsum(w.prefix_len)[:-1]]).astype(np.int64)
-    d["pstart"] = torch.from_numpy(pstart).to(dev)
-    d["plen"] = torch.from_numpy(w.prefix_len).to(dev)
+    d = batch_inputs(w, dev)
     tree = dt.Tree.empty(B, N, V, stochastic=False, device=dev)
     ws_b = dt.workspace(dt.build_workspace_bytes(B, Bk, V, r, kmax, N), dev)
     ws_v = dt.workspace(dt.verify_workspace_bytes(B, N, w.Hq, w.Hkv, w.d, P), dev)
@@ -796,6 +809,127 @@ def run_study(args):
     print(json.dumps(out))
 
 
+LOADS = [1, 2, 4, 8, 16, 32, 64]
+CAPACITY, PREFIX_UNIT = 256, 2048
+
+
+def run_load_policy(args):
+    """Load sweep of the load-adaptive tree size (one GPU).
+
+    At each load (requests per round) the round is built with full N = 32
+    trees, then either verified as built ("fixed") or first cut by
+    dt_tree_load_budget to a verification capacity of CAPACITY units, a node
+    of request b costing 1 + P_b // PREFIX_UNIT units ("adaptive").  Every
+    round is scored by the synthetic first-order target and walked greedily;
+    the headline is the adaptive policy's accepted tokens per second at the
+    highest load."""
+    import torch
+    import draft_tree_construction_markov_b200 as dt
+    from gen import make_workload, target_rows
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    bf = torch.bfloat16
+    w = make_workload("load_sweep", seed=rank)
+    V, Bk, N, r, B = w.V, w.Bk, w.Nmax, w.r, w.batch
+    d = batch_inputs(w, dev)
+    stream = torch.cuda.Stream(device=dev)
+    full = dt.Tree.empty(B, N, V, device=dev)
+    ws_b = dt.workspace(dt.build_workspace_bytes(B, Bk, V, r, w.k, N), dev)
+    with torch.cuda.stream(stream):
+        dt.tree_build(d["L"], d["A"], d["Bt"], d["root"], d["nb"], d["lam"], k=w.k, Nmax=N,
+                      temp=0.0, out=full, ws=ws_b)
+    torch.cuda.synchronize()
+    assert dt.read_status(ws_b) == 0
+    # requests are independent: the first L requests of any build have these
+    # trees, so one set of target rows serves every load
+    n_full = full.n_nodes.cpu().numpy()
+    toks, deps = full.tokens.cpu().numpy(), full.depths.cpu().numpy()
+    tgt = torch.empty(B, N + 1, V, dtype=bf, device=dev)
+    for b in range(B):
+        n = int(n_full[b])
+        rows = target_rows(w, b, np.concatenate([[0], deps[b, :n]]),
+                           np.concatenate([w.root[b:b + 1], toks[b, :n]]))
+        tgt[b, : n + 1].copy_(torch.from_numpy(rows))
+    cost = 1 + w.prefix_len.astype(np.int64) // PREFIX_UNIT
+    rows_out, clocks = [], ClockSampler(local)
+    clocks.start()
+    for Lq in LOADS:
+        P = int(w.prefix_len[:Lq].max())
+        tree = dt.Tree.empty(Lq, N, V, device=dev)
+        ws_v = dt.workspace(dt.verify_workspace_bytes(Lq, N, w.Hq, w.Hkv, w.d, P), dev)
+        ws_a = dt.workspace(dt.accept_workspace_bytes(Lq, N, V), dev)
+        ws_p = dt.workspace(dt.load_budget_workspace_bytes(), dev)
+        attn_out = torch.empty(Lq, N + 1, w.Hq, w.d, dtype=bf, device=dev)
+        acc = torch.empty(Lq, Bk, dtype=torch.int32, device=dev)
+        nacc = torch.empty(Lq, dtype=torch.int32, device=dev)
+        bonus = torch.empty(Lq, dtype=torch.int32, device=dev)
+        s = lambda x: x[:Lq]
+
+        def round_(adaptive):
+            dt.tree_build(s(d["L"]), d["A"], d["Bt"], s(d["root"]), s(d["nb"]), s(d["lam"]),
+                          k=w.k, Nmax=N, temp=0.0, out=tree, ws=ws_b)
+            if adaptive:
+                dt.tree_load_budget(tree, CAPACITY, ws_p, prefix_len=s(d["plen"]),
+                                    prefix_unit=PREFIX_UNIT)
+            dt.tree_verify_attn(s(d["q"]), d["kp"], d["vp"], s(d["pstart"]), s(d["plen"]), P,
+                                s(d["kt"]), s(d["vt"]), tree.anc, tree.n_nodes,
+                                1.0 / math.sqrt(w.d), attn_out, ws_v)
+            dt.tree_accept(s(tgt), tree, Bk, 0.0, acc, nacc, bonus, ws_a)
+
+        for adaptive in (False, True):
+            with torch.cuda.stream(stream):
+                for _ in range(max(args.warmup, 3)):
+                    round_(adaptive)
+            torch.cuda.synchronize()
+            for wsx in (ws_b, ws_v, ws_a) + ((ws_p,) if adaptive else ()):
+                assert dt.read_status(wsx) == 0
+            kept = tree.n_nodes.cpu().numpy()
+            tau = nacc.cpu().numpy() + 1
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                round_(adaptive)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                for _ in range(args.warmup):
+                    g.replay()
+                e0.record(stream)
+                for _ in range(args.steps):
+                    g.replay()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            del g
+            units = int((kept * cost[:Lq]).sum())
+            rows_out.append({
+                "load": Lq, "policy": "adaptive" if adaptive else "fixed",
+                "nodes_per_request": round(float(kept.mean()), 3),
+                "units_used": units,
+                "accept_len": round(float(tau.mean()), 4),
+                # accepted tokens per verified unit (each root row costs one unit too)
+                "tokens_per_unit": round(float(tau.sum()) / (units + int(cost[:Lq].sum())), 4),
+                "ms_per_round": round(ms, 4),
+                "accepted_tokens_per_s": round(float(tau.sum()) / (ms / 1e3), 1)})
+    clk = clocks.stop()
+    head = [x for x in rows_out if x["load"] == LOADS[-1] and x["policy"] == "adaptive"][0]
+    out = {
+        "metric": "accepted tokens per verified unit at 64 requests under a 256-unit round "
+                  "capacity, load-adaptive tree size (build + load budget + verify + accept); "
+                  "load sweep with round times in 'sweep'",
+        "value": head["tokens_per_unit"], "unit": "tokens/unit", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_round"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": DESCS["load_policy"], "capacity_units": CAPACITY,
+                   "prefix_unit": PREFIX_UNIT,
+                   "l2": "Markov factors 156 MB + target rows > 126 MB L2 per round",
+                   "round": "CUDA graph per (load, policy)"},
+        "sweep": rows_out, "clocks": clk,
+    }
+    print(json.dumps(out))
+
+
 def run_reference(args):
     """The oracle as the reference arm: each step is one CPU round of the workload."""
     rank, world, local = dist_env()
@@ -843,5 +977,7 @@ if __name__ == "__main__":
         run_treeflash(a)
     elif a.workload == "acceptance_study":
         run_study(a)
+    elif a.workload == "load_policy":
+        run_load_policy(a)
     else:
         run_ours(a)

@@ -16,7 +16,8 @@ from ._lib import DtreeError, check, dtype_code, ptr, stream_ptr
 
 __all__ = ["Tree", "tree_build", "tree_verify_attn", "tree_accept", "markov_logits",
            "read_status", "build_workspace_bytes", "verify_workspace_bytes",
-           "accept_workspace_bytes", "workspace", "DtreeError", "num_sms"]
+           "accept_workspace_bytes", "workspace", "DtreeError", "num_sms", "tree_load_budget",
+           "load_budget_workspace_bytes"]
 
 
 def num_sms() -> int:
@@ -24,7 +25,11 @@ def num_sms() -> int:
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    """Device scratch for one call site; its 256-byte header (the status word
+    that read_status returns) starts cleared."""
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
 
 
 @dataclass
@@ -141,6 +146,22 @@ def treeflash_build(h, embed, w_norm_h, w_norm_e, w_gate, w_up, w_down, w_lm, ro
         ptr(w_lm), ptr(root), batch, gamma, D, Dff, V, M, budget, ctypes.byref(st), ptr(ws),
         ws.numel(), stream_ptr(stream)), "dt_treeflash_build")
     return out
+
+
+def tree_load_budget(tree: Tree, capacity, ws, *, prefix_len=None, prefix_unit=0, n_keep=None,
+                     stream=None):
+    """dt_tree_load_budget: cut the batch's trees (in place) to a round's
+    verification capacity by survival; returns ``tree``."""
+    batch, Nmax = tree.keys.shape
+    st = tree.c_struct()
+    check(_lib.lib.dt_tree_load_budget(
+        ctypes.byref(st), batch, Nmax, ptr(prefix_len), int(capacity), int(prefix_unit),
+        ptr(n_keep), ptr(ws), ws.numel(), stream_ptr(stream)), "dt_tree_load_budget")
+    return tree
+
+
+def load_budget_workspace_bytes() -> int:
+    return int(_lib.lib.dt_tree_load_budget_workspace_bytes())
 
 
 def read_status(ws, stream=None) -> int:

@@ -59,6 +59,13 @@ CONFIGS = {
                              logit_dtype="bf16", L_scale=3.0, plant=("margin", 8.0, 2.0),
                              target_sigma=1.0, P=1024, Hq=32, Hkv=8, d=128,
                              attn_dtype="bf16", batch=64, temp=0.0, lam=0.0),
+    # Load sweep of the load-adaptive tree size: the acceptance-study block
+    # with lognormal prefixes clipped to [512, 8192] (the load-adaptive
+    # recipe); every request asks for the full N = 32 tree.
+    "load_sweep": dict(V=151936, Bk=16, k=4, N=32, r=256, sigma_ab=0.35,
+                       logit_dtype="bf16", L_scale=3.0, plant=("margin", 8.0, 2.0),
+                       target_sigma=1.0, P=8192, Hq=32, Hkv=8, d=128,
+                       attn_dtype="bf16", batch=64, temp=0.0, lam=0.0, ragged_prefix=True),
     # Load-adaptive batch: 64 requests, lognormal prefixes clipped to
     # [512, 8192], per-request budget from {chain, 8, 16, 32}, lambda 0.01, T=1.
     "load_adaptive": dict(V=151936, Bk=7, k=4, N=32, r=256, sigma_ab=0.25,
@@ -168,6 +175,10 @@ def make_workload(name: str, seed: int = 0, **over) -> Workload:
     gm = rng(seed, _T_META)
     root = gm.integers(0, V, size=batch).astype(np.int32)
     N, k = c["N"], c["k"]
+    if c.get("ragged_prefix"):
+        # lognormal prefixes only (same recipe as the load-adaptive batch)
+        plen_r = np.clip(np.round(1024.0 * np.exp(0.7 * gm.standard_normal(batch))),
+                         512, c["P"]).astype(np.int32)
     if c.get("ragged"):
         # per-request budget drawn from {chain, 8, 16, 32}; chain = k 1, N = Bk
         choice = gm.integers(0, 4, size=batch)
@@ -179,7 +190,7 @@ def make_workload(name: str, seed: int = 0, **over) -> Workload:
     else:
         n_budget = np.full(batch, N, np.int32)
         k_req = np.full(batch, k, np.int32)
-        plen = np.full(batch, c["P"], np.int32)
+        plen = plen_r if c.get("ragged_prefix") else np.full(batch, c["P"], np.int32)
         Nmax = N
     lam = np.full(batch, c["lam"], np.float32)
     return Workload(

@@ -6,6 +6,8 @@
  *                       of drafter logits and a low-rank Markov head
  *   dt_tree_build_ex    the same, or one of the baseline trees it is compared
  *                       with (chain, marginal-ranked, Shared-Markov)
+ *   dt_tree_load_budget cut a batch of trees to a round's verification
+ *                       capacity by survival (load-adaptive tree size)
  *   dt_tree_verify_attn tree-masked grouped-query attention over prefix + tree
  *   dt_tree_accept      lossless acceptance walk (greedy or recursive residual)
  *
@@ -278,6 +280,36 @@ dt_status dt_tree_accept_noalloc(const void* d_target_logits, dt_dtype tdt,
                                  uint64_t philox_offset, int32_t* d_acc_nodes,
                                  int32_t* d_n_acc, int32_t* d_bonus,
                                  dt_stream stream);
+
+/* ---------------------------------------------------------- load policy --
+ * Load-adaptive tree size (TreeSpark article, "core idea": the load-adaptive
+ * serving policy sizes the trees with the same calibrated path survival that
+ * drives expansion and stopping; "measured gains": under rising load the
+ * trees shrink back toward the chain).  Applied to built trees before
+ * verification, it cuts them so that the batch fits a round's verification
+ * capacity:
+ *   - a verified node of request b costs w_b = 1 + floor(P_b / prefix_unit)
+ *     units, P_b = d_prefix_len[b] (NULL or prefix_unit == 0: w_b = 1);
+ *   - the batch's nodes are ordered by (fp32 key desc, request asc, pop index
+ *     asc) and the longest prefix of that order whose total cost is
+ *     <= capacity is kept.
+ * Keys are non-increasing along a tree's pop order, so request b keeps its
+ * first n'_b nodes, an ancestor-closed subtree: d_n_nodes[b] is overwritten
+ * with n'_b (also written to d_n_keep[b] unless NULL); every other tree array
+ * stays valid as it is.  With all nodes fitting nothing changes; capacity 0
+ * leaves every tree empty (the round emits the bonus token only).
+ *   tree      the dt_tree of dt_tree_build (d_keys and d_n_nodes are used)
+ *   limits    1 <= batch <= 1024, 1 <= Nmax <= 64, capacity >= 0,
+ *             prefix_unit >= 0
+ *   ws        >= dt_tree_load_budget_workspace_bytes() bytes (status word)
+ * A node count outside [0, Nmax] or a negative prefix length sets DT_EDEVICE
+ * in the status word. */
+size_t dt_tree_load_budget_workspace_bytes(void);
+
+dt_status dt_tree_load_budget(const dt_tree* tree, int batch, int Nmax,
+                              const int32_t* d_prefix_len, int64_t capacity,
+                              int prefix_unit, int32_t* d_n_keep, void* ws,
+                              size_t ws_bytes, dt_stream stream);
 
 /* Synchronises `stream` and returns the status word that device code of the
  * last call using `ws` wrote (DT_OK, DT_ETIMEOUT or DT_EDEVICE), then clears

@@ -43,6 +43,8 @@ def load_budget(keys, n_nodes, prefix_len, capacity, prefix_unit):
     """
     keys = np.asarray(keys, np.float32)
     n_nodes = np.asarray(n_nodes, np.int64)
+    if prefix_len is None:  # no prefix lengths: every node costs one unit
+        prefix_len = np.zeros(len(n_nodes), np.int64)
     w = node_cost(prefix_len, prefix_unit)
     order = sorted(((-float(keys[b, i]), b, i) for b in range(len(n_nodes))
                     for i in range(int(n_nodes[b]))))
