@@ -21,6 +21,8 @@ variants     the baseline trees of the PCTree summary's mechanism isolation
              (chain, marginal-ranked, Shared-Markov) and acceptance length.
 load_policy  survival-ordered allocation of a round's verification capacity
              over a batch (TreeSpark article, load-adaptive serving policy).
+calibration  logged (depth, log-probability, accepted) triples and the
+             per-depth maximum-likelihood fit of the calibration.
 
 Every floating quantity is fp64; inputs are the exact stored values.
 """
