@@ -17,7 +17,7 @@ from ._lib import DtreeError, check, dtype_code, ptr, stream_ptr
 __all__ = ["Tree", "tree_build", "tree_verify_attn", "tree_accept", "markov_logits",
            "read_status", "build_workspace_bytes", "verify_workspace_bytes",
            "accept_workspace_bytes", "workspace", "DtreeError", "num_sms", "tree_load_budget",
-           "load_budget_workspace_bytes"]
+           "load_budget_workspace_bytes", "calib_workspace_bytes", "calib_log", "calib_fit"]
 
 
 def num_sms() -> int:
@@ -162,6 +162,31 @@ def tree_load_budget(tree: Tree, capacity, ws, *, prefix_len=None, prefix_unit=0
 
 def load_budget_workspace_bytes() -> int:
     return int(_lib.lib.dt_tree_load_budget_workspace_bytes())
+
+
+def calib_workspace_bytes(Bk=1, n_alpha=1, n_beta=1) -> int:
+    return int(_lib.lib.dt_calib_workspace_bytes(Bk, n_alpha, n_beta))
+
+
+def calib_log(tree: Tree, acc_nodes, n_acc, Bk, depth, ell, y, ws, stream=None):
+    """dt_calib_log: (depth, l, y) [batch, Nmax] of every child of a reached node."""
+    batch, Nmax = tree.keys.shape
+    st = tree.c_struct()
+    check(_lib.lib.dt_calib_log(
+        ctypes.byref(st), ptr(acc_nodes), ptr(n_acc), batch, Bk, Nmax, ptr(depth), ptr(ell), ptr(y),
+        ptr(ws), ws.numel(), stream_ptr(stream)), "dt_calib_log")
+    return depth, ell, y
+
+
+def calib_fit(depth, ell, y, Bk, grid, calib, ws, loglik=None, stream=None):
+    """dt_calib_fit over the flattened samples; grid = (alpha0, dalpha, n_alpha,
+    beta0, dbeta, n_beta); writes calib [Bk, 2] fp32 (and loglik [Bk] fp64)."""
+    a0, da, na, b0, db, nb = grid
+    check(_lib.lib.dt_calib_fit(
+        ptr(depth), ptr(ell), ptr(y), depth.numel(), Bk, float(a0), float(da), int(na), float(b0),
+        float(db), int(nb), ptr(calib), ptr(loglik), ptr(ws), ws.numel(), stream_ptr(stream)),
+        "dt_calib_fit")
+    return calib
 
 
 def read_status(ws, stream=None) -> int:

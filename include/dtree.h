@@ -8,6 +8,7 @@
  *                       with (chain, marginal-ranked, Shared-Markov)
  *   dt_tree_load_budget cut a batch of trees to a round's verification
  *                       capacity by survival (load-adaptive tree size)
+ *   dt_calib_log/_fit   log verified rounds and fit the calibration
  *   dt_tree_verify_attn tree-masked grouped-query attention over prefix + tree
  *   dt_tree_accept      lossless acceptance walk (greedy or recursive residual)
  *
@@ -310,6 +311,46 @@ dt_status dt_tree_load_budget(const dt_tree* tree, int batch, int Nmax,
                               const int32_t* d_prefix_len, int64_t capacity,
                               int prefix_unit, int32_t* d_n_keep, void* ws,
                               size_t ws_bytes, dt_stream stream);
+
+/* ---------------------------------------------------------- calibration --
+ * Fitting the calibration c_d(l) = min(0, alpha_d l + beta_d) that
+ * dt_tree_build takes as d_calib (TreeSpark article, "core idea": the
+ * drafter's parent-conditioned probability is calibrated into an estimate of
+ * the edge's acceptance; the pages give no fitting method).
+ *
+ * dt_calib_log logs one greedily verified round: for node i of request b
+ * whose parent the walk reached (the root, or a node of the accepted path
+ * d_acc_nodes[b][0 .. d_n_acc[b]) of dt_tree_accept), it writes
+ *   d_depth[b][i] = depth of i,  d_ell[b][i] = key(i) - key(parent) in fp32
+ *   (key(root) = 0), d_y[b][i] = 1 iff i is on the accepted path;
+ * every other slot of [batch][Nmax] gets depth -1.  With a tree built with
+ * the identity calibration, l is the child's drafter log-probability (the
+ * order statistic of its rank).  Limits: batch <= 1024, Bk <= 16,
+ * Nmax <= 64; ws >= dt_calib_workspace_bytes(1, 1, 1).  Out-of-range counts,
+ * path nodes or parents set DT_EDEVICE.
+ *
+ * dt_calib_fit fits every child depth d = 1..Bk on the n logged samples
+ * (entries with depth outside 1..Bk are ignored): it scans the grid
+ *   alpha_i = alpha0 + i * dalpha (i < n_alpha),
+ *   beta_j = beta0 + j * dbeta (j < n_beta)   (fp64; alpha0, dalpha, dbeta >= 0)
+ * and keeps the point with the largest Bernoulli log-likelihood
+ *   sum_{y=1} c(l) + sum_{y=0} log(1 - exp(c(l))),  c(l) = min(0, alpha l + beta)
+ * computed in fp64 (ties to the smaller i, then the smaller j).  Output:
+ * d_calib [Bk][2] fp32 (alpha, beta), directly usable by dt_tree_build; a
+ * depth without samples gets the identity (1, 0).  d_loglik [Bk] (fp64,
+ * NaN without samples) may be NULL.  Limits: Bk <= 16, n_alpha * n_beta
+ * <= 2^20; ws >= dt_calib_workspace_bytes(Bk, n_alpha, n_beta). */
+size_t dt_calib_workspace_bytes(int Bk, int n_alpha, int n_beta);
+
+dt_status dt_calib_log(const dt_tree* tree, const int32_t* d_acc_nodes,
+                       const int32_t* d_n_acc, int batch, int Bk, int Nmax,
+                       int32_t* d_depth, float* d_ell, int8_t* d_y, void* ws,
+                       size_t ws_bytes, dt_stream stream);
+
+dt_status dt_calib_fit(const int32_t* d_depth, const float* d_ell, const int8_t* d_y,
+                       int n, int Bk, float alpha0, float dalpha, int n_alpha,
+                       float beta0, float dbeta, int n_beta, float* d_calib,
+                       double* d_loglik, void* ws, size_t ws_bytes, dt_stream stream);
 
 /* Synchronises `stream` and returns the status word that device code of the
  * last call using `ws` wrote (DT_OK, DT_ETIMEOUT or DT_EDEVICE), then clears
