@@ -47,6 +47,9 @@ DESCS = {
                     "block B=16, k=4, N=32, Markov rank 256 (sigma 0.35), greedy, lognormal "
                     "prefixes 512..8192; trees cut to 256 verification units per round, a node "
                     "costing 1 + prefix // 2048; synthetic first-order target"),
+    "calibration": ("calibration fitting: acceptance-study drafter and target, 64 requests "
+                    "logged with the identity calibration, fp64 likelihood grid 65 x 97 per "
+                    "depth, 64 held-out requests"),
     "treeflash": ("TreeFlash tree build: SwiGLU AR-approximator d=2560, d_ff=2560, bf16 LM head "
                   "2560x151936, M=4, depth 16 (61 evaluations per request), budget B=16, "
                   "batch 16, T=0"),
@@ -62,7 +65,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--copies", type=int, default=4)
     p.add_argument("--no-oracle", action="store_true", help="skip the cpu_baseline leg")
-    p.add_argument("--workload", default=WORKLOAD, choices=["qwen3_4b", "qwen3_8b", "load_adaptive", "treeflash", "acceptance_study", "load_policy"])
+    p.add_argument("--workload", default=WORKLOAD, choices=["qwen3_4b", "qwen3_8b", "load_adaptive", "treeflash", "acceptance_study", "load_policy", "calibration"])
     return p.parse_args()
 
 
@@ -930,6 +933,129 @@ def run_load_policy(args):
     print(json.dumps(out))
 
 
+CAL_GRID = (0.0, 1 / 32, 65, -1.0, 1 / 32, 97)   # alpha 0..2, beta -1..2
+
+
+def run_calibration(args):
+    """Calibration fitting (one GPU): log the greedy rounds of 64 requests
+    built with the identity calibration, fit (alpha_d, beta_d) per depth on
+    the GPU (timed), then compare identity and fitted calibration on 64
+    held-out requests of the same synthetic drafter and target: log loss of
+    the edge-acceptance estimate on the held-out logged edges, and tree size
+    and acceptance length under a survival stop (lambda)."""
+    import torch
+    import draft_tree_construction_markov_b200 as dt
+    from gen import make_workload, target_rows
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    bf = torch.bfloat16
+    w = make_workload("acceptance_study", seed=rank, batch=128)
+    V, Bk, N, r = w.V, w.Bk, w.Nmax, w.r
+    H = 64  # requests per half
+    cu = lambda a, tt=bf: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(tt)
+    A, Bt = cu(w.A), cu(w.Bt)
+    stream = torch.cuda.Stream(device=dev)
+    ws_b = dt.workspace(dt.build_workspace_bytes(H, Bk, V, r, w.k, N), dev)
+    ws_a = dt.workspace(dt.accept_workspace_bytes(H, N, V), dev)
+    ws_c = dt.workspace(dt.calib_workspace_bytes(Bk, CAL_GRID[2], CAL_GRID[5]), dev)
+    tgt = torch.empty(H, N + 1, V, dtype=bf, device=dev)
+
+    def rounds(lo, calib, lam):
+        """Build, score and walk requests lo..lo+H; logged edges and outcomes."""
+        Lb = cu(w.L[lo:lo + H])
+        root = torch.from_numpy(w.root[lo:lo + H]).to(dev)
+        nb = torch.full((H,), N, dtype=torch.int32, device=dev)
+        lamt = torch.full((H,), lam, dtype=torch.float32, device=dev)
+        tree = dt.Tree.empty(H, N, V, device=dev)
+        with torch.cuda.stream(stream):
+            dt.tree_build(Lb, A, Bt, root, nb, lamt, k=w.k, Nmax=N, temp=0.0, out=tree, ws=ws_b,
+                          calib=calib)
+        torch.cuda.synchronize()
+        assert dt.read_status(ws_b) == 0
+        n = tree.n_nodes.cpu().numpy()
+        toks, deps = tree.tokens.cpu().numpy(), tree.depths.cpu().numpy()
+        for b in range(H):
+            rows = target_rows(w, lo + b, np.concatenate([[0], deps[b, :n[b]]]),
+                               np.concatenate([w.root[lo + b:lo + b + 1], toks[b, :n[b]]]))
+            tgt[b, : n[b] + 1].copy_(torch.from_numpy(rows))
+        acc = torch.empty(H, Bk, dtype=torch.int32, device=dev)
+        nacc = torch.empty(H, dtype=torch.int32, device=dev)
+        bonus = torch.empty(H, dtype=torch.int32, device=dev)
+        dt.tree_accept(tgt, tree, Bk, 0.0, acc, nacc, bonus, ws_a)
+        assert dt.read_status(ws_a) == 0
+        depth = torch.empty(H, N, dtype=torch.int32, device=dev)
+        ell = torch.empty(H, N, dtype=torch.float32, device=dev)
+        y = torch.empty(H, N, dtype=torch.int8, device=dev)
+        dt.calib_log(tree, acc, nacc, Bk, depth, ell, y, ws_c)
+        assert dt.read_status(ws_c) == 0
+        return dict(n=n, tau=nacc.cpu().numpy() + 1, depth=depth, ell=ell, y=y)
+
+    fit_set = rounds(0, None, 0.0)
+    cal = torch.empty(Bk, 2, dtype=torch.float32, device=dev)
+    ll = torch.empty(Bk, dtype=torch.float64, device=dev)
+    dflat, eflat, yflat = (fit_set[x].reshape(-1) for x in ("depth", "ell", "y"))
+    for _ in range(max(args.warmup, 3)):
+        dt.calib_fit(dflat, eflat, yflat, Bk, CAL_GRID, cal, ws_c, loglik=ll)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(args.steps, 1)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            dt.calib_fit(dflat, eflat, yflat, Bk, CAL_GRID, cal, ws_c, loglik=ll, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    assert dt.read_status(ws_c) == 0
+    fit_ms = e0.elapsed_time(e1) / reps
+    calib = cal.clone()
+    n_samples = int((dflat.cpu().numpy() > 0).sum())
+
+    # held-out requests: logged edges of the identity-calibrated trees
+    held = rounds(H, None, 0.0)
+    d_h = held["depth"].cpu().numpy().reshape(-1)
+    l_h = held["ell"].cpu().numpy().reshape(-1).astype(np.float64)
+    y_h = held["y"].cpu().numpy().reshape(-1).astype(bool)
+    m = d_h > 0
+    c_np = calib.cpu().numpy()
+
+    def log_loss(alpha, beta):
+        p = np.exp(np.minimum(0.0, alpha * l_h[m] + beta))
+        p = np.clip(p, 1e-12, 1 - 1e-12)
+        return float(-np.mean(np.where(y_h[m], np.log(p), np.log1p(-p))))
+
+    ident = log_loss(np.ones(m.sum()), np.zeros(m.sum()))
+    fitted = log_loss(c_np[d_h[m] - 1, 0].astype(np.float64), c_np[d_h[m] - 1, 1].astype(np.float64))
+    stops = {}
+    for lam in (0.0, 0.05):
+        for name, cb in (("identity", None), ("fitted", calib)):
+            res = rounds(H, cb, lam)
+            stops[f"{name}_lambda{lam}"] = {
+                "nodes_per_request": round(float(res["n"].mean()), 3),
+                "accept_len": round(float(res["tau"].mean()), 4),
+                "accepted_per_node": round(float((res["tau"] - 1).sum() / max(res["n"].sum(), 1)), 4)}
+    head = stops["fitted_lambda0.05"]
+    out = {
+        "metric": "held-out acceptance length with the GPU-fitted calibration under a survival "
+                  "stop (lambda 0.05, N<=32), acceptance-study config; fit time and log losses "
+                  "in 'calibration'",
+        "value": head["accept_len"], "unit": "tokens/round", "n_gpus": 1, "steps": reps,
+        "warmup": args.warmup, "ms_per_step": round(fit_ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fit), bf16 (rounds)",
+        "data": "synthetic",
+        "config": {"workload": DESCS["calibration"], "grid": list(CAL_GRID)},
+        "calibration": {"fit_ms": round(fit_ms, 4), "fit_samples": n_samples,
+                        "grid_points_per_depth": CAL_GRID[2] * CAL_GRID[5],
+                        "alpha_beta": [[round(float(a), 5), round(float(b), 5)] for a, b in c_np],
+                        "heldout_log_loss_identity": round(ident, 5),
+                        "heldout_log_loss_fitted": round(fitted, 5),
+                        "heldout_edges": int(m.sum())},
+        "stops": stops,
+    }
+    print(json.dumps(out))
+
+
 def run_reference(args):
     """The oracle as the reference arm: each step is one CPU round of the workload."""
     rank, world, local = dist_env()
@@ -979,5 +1105,7 @@ if __name__ == "__main__":
         run_study(a)
     elif a.workload == "load_policy":
         run_load_policy(a)
+    elif a.workload == "calibration":
+        run_calibration(a)
     else:
         run_ours(a)
