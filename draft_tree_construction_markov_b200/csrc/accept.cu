@@ -8,12 +8,19 @@
 // Two launches.  A pre-pass over every target row of every request (row 0 =
 // root, row i+1 = node i, rows past n_nodes skipped) computes, per row chunk,
 // the argmax (T = 0) or the max and sum of exp(t / T) (T > 0).  The walk then
-// runs one CTA per request: at T = 0 it only compares child tokens with row
-// argmaxes; at T > 0 every rejected sibling costs one vocabulary-wide residual
-// pass, r <- max(p - q_j, 0), done by the whole CTA with 128-bit loads.
+// runs one warp per request at T = 0, where it only compares child tokens
+// with row argmaxes, and one thread-block cluster per request at T > 0, where
+// every rejected sibling costs one vocabulary-wide residual pass,
+// r <- max(p - q_j, 0), split over the cluster's CTAs.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace dt {
+
+int num_sms();  // SMs of the current device (api_build.cu)
 
 constexpr int kPreThreads = 256;
 constexpr int kWalkThreads = 1024;
@@ -236,9 +243,48 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return red[0];
 }
 
-// Stochastic walk, one CTA per request.
+// Stochastic walk, one thread-block cluster per request.  The C CTAs of the
+// cluster own consecutive slices of the vocabulary; a residual pass or the
+// bonus race runs over all slices at once, and its sums (or arg-max) are
+// combined through distributed shared memory in a fixed order, so every CTA
+// of the cluster holds the same totals and takes the same decisions.  A
+// child's p(x) and q(x) are read from global memory by every CTA (the
+// residual written by the slice's owner is visible after the cluster barrier
+// of the reduction that followed it).
+struct __align__(8) WalkPart {
+  float a, b;
+};
+
+// Totals of (a, b) over the cluster, identical in every thread of every CTA:
+// block sums, then the CTAs' values combined by one fixed shuffle tree.
+// `slot` alternates between consecutive calls, so a slot is rewritten only
+// after a later cluster barrier has ordered every peer's read of it.
+__device__ __forceinline__ WalkPart cluster_sum2(cg::cluster_group& cl, float a, float b,
+                                                 WalkPart* xs, int slot, float* red,
+                                                 WalkPart* bcast) {
+  a = block_sum<kWalkThreads>(a, red);
+  b = block_sum<kWalkThreads>(b, red);
+  if (threadIdx.x == 0) xs[slot] = WalkPart{a, b};
+  cl.sync();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    WalkPart v{0.f, 0.f};
+    if (lane < (int)cl.num_blocks()) v = *cl.map_shared_rank(&xs[slot], lane);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      v.a += __shfl_xor_sync(0xffffffffu, v.a, o);
+      v.b += __shfl_xor_sync(0xffffffffu, v.b, o);
+    }
+    if (lane == 0) *bcast = v;
+  }
+  __syncthreads();
+  return *bcast;
+}
+
 __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
-  const int b = blockIdx.x;
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  const int b = blockIdx.x / C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ float red[32];
   __shared__ int32_t redi[32];
@@ -246,9 +292,12 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
   __shared__ int s_nk, s_acc;
   __shared__ float s_lse;
   __shared__ int32_t s_tok[64], s_par[64], s_rank[64];
+  __shared__ WalkPart xs[2], bcast;
+  __shared__ float x_best;
+  __shared__ int32_t x_bid;
   int n = w.n_nodes[b];
   if (n < 0 || n > w.Nmax) {
-    if (tid == 0) set_status(w.status, DT_EDEVICE);
+    if (tid == 0 && rank == 0) set_status(w.status, DT_EDEVICE);
     n = n < 0 ? 0 : w.Nmax;
   }
   for (int i = tid; i < n; i += kWalkThreads) {
@@ -258,9 +307,11 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
   }
   __syncthreads();
   const int V = w.V;
+  const int chunk = (V + C - 1) / C;
+  const int v0 = min(V, rank * chunk), v1 = min(V, v0 + chunk);  // this CTA's slice
   const float temp = w.temp;
   float* rb[2] = {w.rbuf + (size_t)b * 2 * V, w.rbuf + (size_t)b * 2 * V + V};
-  int node = -1, nacc = 0;
+  int node = -1, nacc = 0, slot = 0;
   int32_t bonus = 0;
   while (true) {
     const int row = node + 1;
@@ -275,23 +326,23 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
         if (mv != -INFINITY) s2 += w.parts.ps[rg * w.splits + s] * exp2f((mv - m2) * kL2e);
       }
       s2 = warp_sum(s2);
-    if (lane == 0) {
-      s_lse = m2 + logf(s2);
-      int c = 0;
-      for (int i = 0; i < n; ++i)
-        if (s_par[i] == node) kids[c++] = i;
-      for (int i = 1; i < c; ++i) {  // insertion sort by rank (at most k entries)
-        const int v = kids[i];
-        int j = i - 1;
-        while (j >= 0 && s_rank[kids[j]] > s_rank[v]) {
-          kids[j + 1] = kids[j];
-          --j;
+      if (lane == 0) {
+        s_lse = m2 + logf(s2);
+        int c = 0;
+        for (int i = 0; i < n; ++i)
+          if (s_par[i] == node) kids[c++] = i;
+        for (int i = 1; i < c; ++i) {  // insertion sort by rank (at most k entries)
+          const int v = kids[i];
+          int j = i - 1;
+          while (j >= 0 && s_rank[kids[j]] > s_rank[v]) {
+            kids[j + 1] = kids[j];
+            --j;
+          }
+          kids[j + 1] = v;
         }
-        kids[j + 1] = v;
+        s_nk = c;
+        s_acc = -1;
       }
-      s_nk = c;
-      s_acc = -1;
-    }
     }
     __syncthreads();
     const float lse_t = s_lse;
@@ -312,13 +363,14 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
       const float u = philox_uniform(w.seed, w.offset, 1u, (uint32_t)b, (uint32_t)c, 0u, 0u);
       if (u < px / qx) {
         if (tid == 0) s_acc = c;
-        break;  // uniform decision: every thread computed the same values
+        break;  // uniform over the cluster: every thread computed the same values
       }
-      // residual pass: r'(y) = max(p(y) - q_j(y), 0), q_j = q without removed tokens / qn
+      // residual pass over this CTA's slice: r'(y) = max(p(y) - q_j(y), 0),
+      // q_j = q without the tokens removed before x, over the normaliser qn
       removed[n_removed++] = x;
       float* dst = rb[cur ^ 1];
       float zsum = 0.f, qsum = 0.f;
-      for (int y = tid; y < V; y += kWalkThreads) {
+      for (int y = v0 + tid; y < v1; y += kWalkThreads) {
         const float py =
             resid ? rb[cur][y] / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + y), temp) - lse_t);
         bool rm = false;
@@ -330,29 +382,28 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
         zsum += rv;
         if (!rm) qsum += qy;
       }
-      zsum = block_sum<kWalkThreads>(zsum, red);
-      qsum = block_sum<kWalkThreads>(qsum, red);
-      if (zsum > 0.f) {
+      const WalkPart tot = cluster_sum2(cl, zsum, qsum, xs, slot, red, &bcast);
+      slot ^= 1;
+      if (tot.a > 0.f) {
         cur ^= 1;
-        zr = zsum;
+        zr = tot.a;
         resid = true;
       }
-      qn = qsum;
-      __syncthreads();
+      qn = tot.b;
     }
     __syncthreads();
     const int acc = s_acc;
     if (acc >= 0 && nacc < w.Bk) {
-      if (tid == 0) w.acc_nodes[(size_t)b * w.Bk + nacc] = acc;
+      if (tid == 0 && rank == 0) w.acc_nodes[(size_t)b * w.Bk + nacc] = acc;
       ++nacc;
       node = acc;
       __syncthreads();
       continue;
     }
-    // bonus: exponential race argmax_y p(y) / E_y
+    // bonus: exponential race argmax_y p(y) / E_y over every slice
     float best = -INFINITY;
     int32_t bid = 0x7fffffff;
-    for (int y = tid; y < V; y += kWalkThreads) {
+    for (int y = v0 + tid; y < v1; y += kWalkThreads) {
       const float py =
           resid ? rb[cur][y] / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + y), temp) - lse_t);
       const float u = philox_uniform(w.seed, w.offset, 2u, (uint32_t)b, (uint32_t)(node + 1), 0u,
@@ -383,15 +434,37 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
           best = red[i];
           bid = redi[i];
         }
-      bonus = bid;
+      x_best = best;
+      x_bid = bid;
+    }
+    cl.sync();
+    if (tid < 32) {
+      float vb = -INFINITY;
+      int32_t vi = 0x7fffffff;
+      if (lane < C) {
+        vb = *cl.map_shared_rank(&x_best, lane);
+        vi = *cl.map_shared_rank(&x_bid, lane);
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, vb, o);
+        const int32_t oi = __shfl_xor_sync(0xffffffffu, vi, o);
+        if (ov > vb || (ov == vb && oi < vi)) {
+          vb = ov;
+          vi = oi;
+        }
+      }
+      bonus = vi;
     }
     break;
   }
-  if (tid == 0) {
+  if (tid == 0 && rank == 0) {
     for (int i = nacc; i < w.Bk; ++i) w.acc_nodes[(size_t)b * w.Bk + i] = -1;
     w.n_acc[b] = nacc;
     w.bonus[b] = bonus;
   }
+  // no CTA leaves while a peer may still read its shared memory
+  cl.sync();
 }
 
 }  // namespace dt
@@ -482,10 +555,27 @@ dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt, const dt_tre
   w.bonus = d_bonus;
   w.status = status;
   ProfileScope ps(DT_K_ACCEPT_WALK, s);
-  if (temp > 0.f)
-    stoch_walk_kernel<<<batch, kWalkThreads, 0, s>>>(w);
-  else
+  if (temp > 0.f) {
+    // one cluster of C CTAs per request: as many as keep every request's
+    // cluster resident at once (one 1024-thread CTA per SM), at most 8
+    int C = 8;
+    while (C > 1 && (long long)batch * C > num_sms()) C >>= 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(batch * C);
+    cfg.blockDim = dim3(kWalkThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, stoch_walk_kernel, w) != cudaSuccess) return DT_ECUDA;
+  } else {
     greedy_walk_kernel<<<batch, 32, 0, s>>>(w);
+  }
   if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
   return DT_OK;
 }
