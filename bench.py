@@ -47,9 +47,9 @@ DESCS = {
                     "block B=16, k=4, N=32, Markov rank 256 (sigma 0.35), greedy, lognormal "
                     "prefixes 512..8192; trees cut to 256 verification units per round, a node "
                     "costing 1 + prefix // 2048; synthetic first-order target"),
-    "calibration": ("calibration fitting: acceptance-study drafter and target, 64 requests "
+    "calibration": ("calibration fitting: acceptance-study drafter and target, 192 requests "
                     "logged with the identity calibration, fp64 likelihood grid 65 x 97 per "
-                    "depth, 64 held-out requests"),
+                    "depth (depths with >= 100 logged edges), 64 held-out requests"),
     "treeflash": ("TreeFlash tree build: SwiGLU AR-approximator d=2560, d_ff=2560, bf16 LM head "
                   "2560x151936, M=4, depth 16 (61 evaluations per request), budget B=16, "
                   "batch 16, T=0"),
@@ -934,6 +934,7 @@ def run_load_policy(args):
 
 
 CAL_GRID = (0.0, 1 / 32, 65, -1.0, 1 / 32, 97)   # alpha 0..2, beta -1..2
+CAL_MIN = 100  # logged edges a depth needs to be fitted
 
 
 def run_calibration(args):
@@ -951,9 +952,9 @@ def run_calibration(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     bf = torch.bfloat16
-    w = make_workload("acceptance_study", seed=rank, batch=128)
+    F, H = 3, 64  # fit on F rounds of H requests, hold out the next H
+    w = make_workload("acceptance_study", seed=rank, batch=(F + 1) * H)
     V, Bk, N, r = w.V, w.Bk, w.Nmax, w.r
-    H = 64  # requests per half
     cu = lambda a, tt=bf: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(tt)
     A, Bt = cu(w.A), cu(w.Bt)
     stream = torch.cuda.Stream(device=dev)
@@ -992,19 +993,22 @@ def run_calibration(args):
         assert dt.read_status(ws_c) == 0
         return dict(n=n, tau=nacc.cpu().numpy() + 1, depth=depth, ell=ell, y=y)
 
-    fit_set = rounds(0, None, 0.0)
+    fit_sets = [rounds(f * H, None, 0.0) for f in range(F)]
     cal = torch.empty(Bk, 2, dtype=torch.float32, device=dev)
     ll = torch.empty(Bk, dtype=torch.float64, device=dev)
-    dflat, eflat, yflat = (fit_set[x].reshape(-1) for x in ("depth", "ell", "y"))
+    dflat, eflat, yflat = (torch.cat([fs[x].reshape(-1) for fs in fit_sets])
+                           for x in ("depth", "ell", "y"))
     for _ in range(max(args.warmup, 3)):
-        dt.calib_fit(dflat, eflat, yflat, Bk, CAL_GRID, cal, ws_c, loglik=ll)
+        dt.calib_fit(dflat, eflat, yflat, Bk, CAL_GRID, cal, ws_c, loglik=ll,
+                     min_samples=CAL_MIN)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     reps = max(args.steps, 1)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(reps):
-            dt.calib_fit(dflat, eflat, yflat, Bk, CAL_GRID, cal, ws_c, loglik=ll, stream=stream)
+            dt.calib_fit(dflat, eflat, yflat, Bk, CAL_GRID, cal, ws_c, loglik=ll,
+                         min_samples=CAL_MIN, stream=stream)
         e1.record(stream)
     torch.cuda.synchronize()
     assert dt.read_status(ws_c) == 0
@@ -1013,7 +1017,7 @@ def run_calibration(args):
     n_samples = int((dflat.cpu().numpy() > 0).sum())
 
     # held-out requests: logged edges of the identity-calibrated trees
-    held = rounds(H, None, 0.0)
+    held = rounds(F * H, None, 0.0)
     d_h = held["depth"].cpu().numpy().reshape(-1)
     l_h = held["ell"].cpu().numpy().reshape(-1).astype(np.float64)
     y_h = held["y"].cpu().numpy().reshape(-1).astype(bool)
@@ -1030,7 +1034,7 @@ def run_calibration(args):
     stops = {}
     for lam in (0.0, 0.05):
         for name, cb in (("identity", None), ("fitted", calib)):
-            res = rounds(H, cb, lam)
+            res = rounds(F * H, cb, lam)
             stops[f"{name}_lambda{lam}"] = {
                 "nodes_per_request": round(float(res["n"].mean()), 3),
                 "accept_len": round(float(res["tau"].mean()), 4),
@@ -1046,6 +1050,9 @@ def run_calibration(args):
         "data": "synthetic",
         "config": {"workload": DESCS["calibration"], "grid": list(CAL_GRID)},
         "calibration": {"fit_ms": round(fit_ms, 4), "fit_samples": n_samples,
+                        "min_samples_per_depth": CAL_MIN,
+                        "samples_per_depth": np.bincount(dflat.cpu().numpy()[
+                            dflat.cpu().numpy() > 0], minlength=Bk + 1)[1:].tolist(),
                         "grid_points_per_depth": CAL_GRID[2] * CAL_GRID[5],
                         "alpha_beta": [[round(float(a), 5), round(float(b), 5)] for a, b in c_np],
                         "heldout_log_loss_identity": round(ident, 5),

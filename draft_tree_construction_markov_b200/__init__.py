@@ -178,14 +178,14 @@ def calib_log(tree: Tree, acc_nodes, n_acc, Bk, depth, ell, y, ws, stream=None):
     return depth, ell, y
 
 
-def calib_fit(depth, ell, y, Bk, grid, calib, ws, loglik=None, stream=None):
+def calib_fit(depth, ell, y, Bk, grid, calib, ws, loglik=None, min_samples=1, stream=None):
     """dt_calib_fit over the flattened samples; grid = (alpha0, dalpha, n_alpha,
     beta0, dbeta, n_beta); writes calib [Bk, 2] fp32 (and loglik [Bk] fp64)."""
     a0, da, na, b0, db, nb = grid
     check(_lib.lib.dt_calib_fit(
         ptr(depth), ptr(ell), ptr(y), depth.numel(), Bk, float(a0), float(da), int(na), float(b0),
-        float(db), int(nb), ptr(calib), ptr(loglik), ptr(ws), ws.numel(), stream_ptr(stream)),
-        "dt_calib_fit")
+        float(db), int(nb), int(min_samples), ptr(calib), ptr(loglik), ptr(ws), ws.numel(),
+        stream_ptr(stream)), "dt_calib_fit")
     return calib
 
 

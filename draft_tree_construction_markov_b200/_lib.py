@@ -64,8 +64,8 @@ _sig("dt_tree_load_budget", _i32, ctypes.POINTER(DtTree), _i32, _i32, _vp, ctype
 _sig("dt_calib_workspace_bytes", _sz, _i32, _i32, _i32)
 _sig("dt_calib_log", _i32, ctypes.POINTER(DtTree), _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
      _sz, _vp)
-_sig("dt_calib_fit", _i32, _vp, _vp, _vp, _i32, _i32, _f32, _f32, _i32, _f32, _f32, _i32, _vp, _vp,
-     _vp, _sz, _vp)
+_sig("dt_calib_fit", _i32, _vp, _vp, _vp, _i32, _i32, _f32, _f32, _i32, _f32, _f32, _i32, _i32,
+     _vp, _vp, _vp, _sz, _vp)
 _sig("dt_read_status", _i32, _vp, _vp, ctypes.POINTER(ctypes.c_int32))
 _sig("dt_set_profile_events", None, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int32),
      _i32, ctypes.POINTER(ctypes.c_int32))

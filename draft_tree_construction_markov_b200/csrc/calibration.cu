@@ -192,7 +192,8 @@ __global__ void __launch_bounds__(kFitThreads)
 // One thread per depth: the best of its blocks, in block order.
 __global__ void calib_fit_pick_kernel(const FitPartial* __restrict__ part, int nblk, int Bk,
                                       double a0, double da, double b0, double db, int nb,
-                                      float* __restrict__ calib, double* __restrict__ loglik) {
+                                      int min_samples, float* __restrict__ calib,
+                                      double* __restrict__ loglik) {
   const int d = blockIdx.x * blockDim.x + threadIdx.x;
   if (d >= Bk) return;
   double best = -INFINITY;
@@ -206,8 +207,8 @@ __global__ void calib_fit_pick_kernel(const FitPartial* __restrict__ part, int n
       bidx = p.idx;
     }
   }
-  if (seen == 0 || bidx == 0x7fffffff) {
-    calib[2 * d] = 1.f;  // no data at this depth: identity
+  if (seen < min_samples || bidx == 0x7fffffff) {
+    calib[2 * d] = 1.f;  // too few logged edges at this depth: identity
     calib[2 * d + 1] = 0.f;
     if (loglik) loglik[d] = NAN;
   } else {
@@ -253,9 +254,10 @@ dt_status dt_calib_log(const dt_tree* tree, const int32_t* d_acc_nodes, const in
 
 dt_status dt_calib_fit(const int32_t* d_depth, const float* d_ell, const int8_t* d_y, int n,
                        int Bk, float alpha0, float dalpha, int n_alpha, float beta0,
-                       float dbeta, int n_beta, float* d_calib, double* d_loglik, void* ws,
-                       size_t ws_bytes, dt_stream stream) {
+                       float dbeta, int n_beta, int min_samples, float* d_calib,
+                       double* d_loglik, void* ws, size_t ws_bytes, dt_stream stream) {
   if (!d_calib || (n > 0 && (!d_depth || !d_ell || !d_y))) return DT_EINVAL;
+  min_samples = min_samples < 1 ? 1 : min_samples;
   if (n < 0 || Bk < 1 || n_alpha < 1 || n_beta < 1) return DT_EINVAL;
   if (!(alpha0 >= 0.f) || !(dalpha >= 0.f) || !(dbeta >= 0.f) || !(beta0 == beta0))
     return DT_EINVAL;
@@ -274,8 +276,8 @@ dt_status dt_calib_fit(const int32_t* d_depth, const float* d_ell, const int8_t*
   }
   ProfileScope ps(DT_K_OTHER, s);
   calib_fit_pick_kernel<<<1, 32, 0, s>>>(part, nblk, Bk, (double)alpha0, (double)dalpha,
-                                         (double)beta0, (double)dbeta, n_beta, d_calib,
-                                         d_loglik);
+                                         (double)beta0, (double)dbeta, n_beta, min_samples,
+                                         d_calib, d_loglik);
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ECUDA;
 }
 

@@ -337,8 +337,8 @@ dt_status dt_tree_load_budget(const dt_tree* tree, int batch, int Nmax,
  *   sum_{y=1} c(l) + sum_{y=0} log(1 - exp(c(l))),  c(l) = min(0, alpha l + beta)
  * computed in fp64 (ties to the smaller i, then the smaller j).  Output:
  * d_calib [Bk][2] fp32 (alpha, beta), directly usable by dt_tree_build; a
- * depth without samples gets the identity (1, 0).  d_loglik [Bk] (fp64,
- * NaN without samples) may be NULL.  Limits: Bk <= 16, n_alpha * n_beta
+ * depth with fewer than max(1, min_samples) samples keeps the identity
+ * (1, 0).  d_loglik [Bk] (fp64, NaN where the identity is kept) may be NULL.  Limits: Bk <= 16, n_alpha * n_beta
  * <= 2^20; ws >= dt_calib_workspace_bytes(Bk, n_alpha, n_beta). */
 size_t dt_calib_workspace_bytes(int Bk, int n_alpha, int n_beta);
 
@@ -349,8 +349,9 @@ dt_status dt_calib_log(const dt_tree* tree, const int32_t* d_acc_nodes,
 
 dt_status dt_calib_fit(const int32_t* d_depth, const float* d_ell, const int8_t* d_y,
                        int n, int Bk, float alpha0, float dalpha, int n_alpha,
-                       float beta0, float dbeta, int n_beta, float* d_calib,
-                       double* d_loglik, void* ws, size_t ws_bytes, dt_stream stream);
+                       float beta0, float dbeta, int n_beta, int min_samples,
+                       float* d_calib, double* d_loglik, void* ws, size_t ws_bytes,
+                       dt_stream stream);
 
 /* Synchronises `stream` and returns the status word that device code of the
  * last call using `ws` wrote (DT_OK, DT_ETIMEOUT or DT_EDEVICE), then clears

@@ -23,8 +23,9 @@ Readings fixed here:
   * fit: per depth, the grid point (alpha_i = a0 + i*da, beta_j = b0 + j*db)
     with the largest Bernoulli log-likelihood
         sum_y=1 c(l) + sum_y=0 log(1 - exp(c(l)))
-    (ties to the smaller i, then the smaller j); a depth without data keeps
-    the identity (1, 0).
+    (ties to the smaller i, then the smaller j); a depth with fewer than
+    min_samples logged edges (at least one) keeps the identity (1, 0): a
+    handful of edges at a deep level would otherwise fit an estimate of 1.
 """
 from __future__ import annotations
 
@@ -62,15 +63,15 @@ def log_likelihood(alpha, beta, ell, y):
         return float(x[y].sum() + np.log1p(-np.exp(x[~y])).sum())
 
 
-def fit(depth, ell, y, Bk, a0, da, na, b0, db, nb):
+def fit(depth, ell, y, Bk, a0, da, na, b0, db, nb, min_samples=1):
     """(Bk, 2) fitted (alpha, beta) per child depth 1..Bk, and the (Bk,)
-    maximal log-likelihoods (nan where a depth has no data)."""
+    maximal log-likelihoods (nan where a depth keeps the identity)."""
     depth = np.asarray(depth)
     out = np.tile(np.array([1.0, 0.0]), (Bk, 1))
     best_ll = np.full(Bk, np.nan)
     for d in range(1, Bk + 1):
         m = depth == d
-        if not m.any():
+        if m.sum() < max(1, min_samples):
             continue
         best = None
         for i in range(na):

@@ -24,19 +24,20 @@ if torch.cuda.is_available():
 GRID = (0.0, 1 / 16, 33, -1.0, 1 / 16, 25)
 
 
-def _gpu_fit(depth, ell, y, Bk, grid=GRID):
+def _gpu_fit(depth, ell, y, Bk, grid=GRID, min_samples=1):
     cal = torch.empty(Bk, 2, dtype=torch.float32, device="cuda")
     ll = torch.empty(Bk, dtype=torch.float64, device="cuda")
     ws = dt.workspace(dt.calib_workspace_bytes(Bk, grid[2], grid[5]))
     dt.calib_fit(dev(np.asarray(depth, np.int32)), dev(np.asarray(ell, np.float32)),
-                 dev(np.asarray(y, np.int8)), Bk, grid, cal, ws, loglik=ll)
+                 dev(np.asarray(y, np.int8)), Bk, grid, cal, ws, loglik=ll,
+                 min_samples=min_samples)
     assert dt.read_status(ws) == 0
     return cal.cpu().numpy(), ll.cpu().numpy()
 
 
-def _check_fit(depth, ell, y, Bk, grid=GRID):
-    got, got_ll = _gpu_fit(depth, ell, y, Bk, grid)
-    want, want_ll = calibration.fit(depth, ell, y, Bk, *grid)
+def _check_fit(depth, ell, y, Bk, grid=GRID, min_samples=1):
+    got, got_ll = _gpu_fit(depth, ell, y, Bk, grid, min_samples)
+    want, want_ll = calibration.fit(depth, ell, y, Bk, *grid, min_samples=min_samples)
     for d in range(Bk):
         if np.isnan(want_ll[d]):
             assert np.isnan(got_ll[d]) and got[d].tolist() == [1.0, 0.0]
@@ -51,8 +52,10 @@ def _check_fit(depth, ell, y, Bk, grid=GRID):
             assert abs(got_ll[d] - want_ll[d]) <= 1e-9 * max(1.0, abs(want_ll[d]))
 
 
-@pytest.mark.parametrize("seed,n,Bk", [(0, 500, 3), (1, 5000, 7), (2, 20000, 16), (3, 1, 2)])
-def test_fit_matches_oracle(seed, n, Bk):
+@pytest.mark.parametrize("seed,n,Bk,min_samples", [(0, 500, 3, 1), (1, 5000, 7, 1),
+                                                    (2, 20000, 16, 1), (3, 1, 2, 1),
+                                                    (4, 3000, 16, 190)])
+def test_fit_matches_oracle(seed, n, Bk, min_samples):
     g = np.random.default_rng(seed)
     depth = g.integers(0, Bk + 2, n).astype(np.int32)   # includes ignored depths 0, Bk+1
     a_true = g.uniform(0.3, 1.8, Bk + 2)
@@ -60,7 +63,7 @@ def test_fit_matches_oracle(seed, n, Bk):
     ell = g.uniform(-6, 0, n).astype(np.float32)
     p = np.exp(np.minimum(0, a_true[depth] * ell + b_true[depth]))
     y = (g.random(n) < p).astype(np.int8)
-    _check_fit(depth, ell, y, Bk)
+    _check_fit(depth, ell, y, Bk, min_samples=min_samples)
 
 
 def test_fit_degenerate_outcomes():

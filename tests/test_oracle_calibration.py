@@ -7,7 +7,8 @@
   * the likelihood at the chosen point is the maximum of a brute-force scan
     over a finer grid restricted to the same points, and flat likelihoods
     resolve to the smallest alpha, then the smallest beta;
-  * a depth without data keeps the identity.
+  * a depth without data, or with fewer than min_samples edges, keeps the
+    identity.
 A planted sign error in the likelihood (log p for rejections) or a swapped
 (alpha, beta) would miss the recovery pins.
 """
@@ -80,3 +81,15 @@ def test_fit_is_the_grid_maximum_and_breaks_ties_low():
     ell1 = np.linspace(-1, 0, 50).astype(np.float32)
     cal1, ll1 = calibration.fit(np.ones(50, np.int32), ell1, np.ones(50, np.int8), 1, **GRID)
     assert ll1[0] == 0.0 and cal1[0].tolist() == [0.0, 0.0]
+
+
+def test_min_samples_keeps_the_identity():
+    g = np.random.default_rng(21)
+    ell, y = _draw(g, 2000, 0.7, -0.3)
+    depth = np.concatenate([np.ones(1990, np.int32), np.full(10, 2, np.int32)])
+    full, _ = calibration.fit(depth, ell, y, 2, **GRID)
+    cut, ll = calibration.fit(depth, ell, y, 2, **GRID, min_samples=11)
+    assert np.array_equal(cut[0], full[0])            # 1990 edges: fitted as before
+    assert cut[1].tolist() == [1.0, 0.0] and np.isnan(ll[1])
+    same, _ = calibration.fit(depth, ell, y, 2, **GRID, min_samples=10)
+    assert np.array_equal(same, full)
