@@ -17,7 +17,10 @@ from ._lib import DtreeError, check, dtype_code, ptr, stream_ptr
 __all__ = ["Tree", "tree_build", "tree_verify_attn", "tree_accept", "markov_logits",
            "read_status", "build_workspace_bytes", "verify_workspace_bytes",
            "accept_workspace_bytes", "workspace", "DtreeError", "num_sms", "tree_load_budget",
-           "load_budget_workspace_bytes", "calib_workspace_bytes", "calib_log", "calib_fit"]
+           "load_budget_workspace_bytes", "calib_workspace_bytes", "calib_log", "calib_fit",
+           "shard_range", "shard_cfg", "sharded_workspace_bytes", "sharded_partials_bytes",
+           "sharded_build_begin", "sharded_build_gemm", "sharded_build_frontier",
+           "tree_build_sharded"]
 
 
 def num_sms() -> int:
@@ -187,6 +190,68 @@ def calib_fit(depth, ell, y, Bk, grid, calib, ws, loglik=None, min_samples=1, st
         float(db), int(nb), int(min_samples), ptr(calib), ptr(loglik), ptr(ws), ws.numel(),
         stream_ptr(stream)), "dt_calib_fit")
     return calib
+
+
+# ------------------------------------------------ vocabulary-sharded build --
+def shard_range(V, world, rank):
+    """(v_base, v_len): the Markov-factor rows Bm[v_base : v_base + v_len] rank holds."""
+    a, b = ctypes.c_int(0), ctypes.c_int(0)
+    _lib.lib.dt_shard_range(V, world, rank, ctypes.byref(a), ctypes.byref(b))
+    return a.value, b.value
+
+
+def shard_cfg(batch, Bk, V, r, k, Nmax, world, ncta=None):
+    ncta = int(_lib.lib.dt_shard_ncta(V, world)) if ncta is None else ncta
+    return _lib.ShardCfg(batch, Bk, V, r, k, Nmax, world, ncta)
+
+
+def sharded_workspace_bytes(cfg) -> int:
+    return int(_lib.lib.dt_sharded_workspace_bytes(ctypes.byref(cfg)))
+
+
+def sharded_partials_bytes(cfg) -> int:
+    return int(_lib.lib.dt_sharded_partials_bytes(ctypes.byref(cfg)))
+
+
+def sharded_build_begin(cfg, root_token, n_budget, lam, out: Tree, ws, k_req=None, stream=None):
+    st = out.c_struct()
+    check(_lib.lib.dt_sharded_build_begin(
+        ctypes.byref(cfg), ptr(root_token), ptr(n_budget), ptr(k_req), ptr(lam), ctypes.byref(st),
+        ptr(ws), ws.numel(), stream_ptr(stream)), "dt_sharded_build_begin")
+
+
+def sharded_build_gemm(cfg, wave, rank, block_logits, markov_a, markov_b_shard, ws, partials,
+                       stream=None):
+    check(_lib.lib.dt_sharded_build_gemm(
+        ctypes.byref(cfg), wave, rank, ptr(block_logits), dtype_code(block_logits), ptr(markov_a),
+        ptr(markov_b_shard), ptr(ws), ws.numel(), ptr(partials), stream_ptr(stream)),
+        "dt_sharded_build_gemm")
+
+
+def sharded_build_frontier(cfg, wave, gathered, n_budget, lam, out: Tree, ws, calib=None,
+                           k_req=None, stream=None):
+    st = out.c_struct()
+    check(_lib.lib.dt_sharded_build_frontier(
+        ctypes.byref(cfg), wave, ptr(gathered), ptr(calib), ptr(n_budget), ptr(k_req), ptr(lam),
+        ctypes.byref(st), ptr(ws), ws.numel(), stream_ptr(stream)), "dt_sharded_build_frontier")
+
+
+def tree_build_sharded(cfg, rank, block_logits, markov_a, markov_b_shard, root_token, n_budget,
+                       lam, out: Tree, ws, partials, gathered, all_gather, calib=None, k_req=None,
+                       stream=None):
+    """The sharded build's wave loop on one rank.  ``partials`` holds this
+    rank's block (sharded_partials_bytes), ``gathered`` world blocks;
+    ``all_gather(gathered, partials)`` must fill ``gathered`` with every
+    rank's block in rank order (torch.distributed.all_gather_into_tensor over
+    the ranks sharing the vocabulary)."""
+    sharded_build_begin(cfg, root_token, n_budget, lam, out, ws, k_req=k_req, stream=stream)
+    for wave in range(cfg.Bk):
+        sharded_build_gemm(cfg, wave, rank, block_logits, markov_a, markov_b_shard, ws, partials,
+                           stream=stream)
+        all_gather(gathered, partials)
+        sharded_build_frontier(cfg, wave, gathered, n_budget, lam, out, ws, calib=calib,
+                               k_req=k_req, stream=stream)
+    return out
 
 
 def read_status(ws, stream=None) -> int:

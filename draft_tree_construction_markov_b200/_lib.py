@@ -33,6 +33,11 @@ class DtTree(ctypes.Structure):
                 ("d_keys", _vp), ("d_anc", _vp), ("d_n_nodes", _vp), ("d_draft_q", _vp)]
 
 
+class ShardCfg(ctypes.Structure):
+    _fields_ = [(nm, ctypes.c_int) for nm in ("batch", "Bk", "V", "r", "k", "Nmax", "world",
+                                               "ncta")]
+
+
 def _sig(name, restype, *args):
     f = getattr(lib, name)
     f.restype = restype
@@ -66,6 +71,15 @@ _sig("dt_calib_log", _i32, ctypes.POINTER(DtTree), _vp, _vp, _i32, _i32, _i32, _
      _sz, _vp)
 _sig("dt_calib_fit", _i32, _vp, _vp, _vp, _i32, _i32, _f32, _f32, _i32, _f32, _f32, _i32, _i32,
      _vp, _vp, _vp, _sz, _vp)
+_PC = ctypes.POINTER(ShardCfg)
+_sig("dt_shard_range", None, _i32, _i32, _i32, ctypes.POINTER(_i32), ctypes.POINTER(_i32))
+_sig("dt_shard_ncta", _i32, _i32, _i32)
+_sig("dt_sharded_workspace_bytes", _sz, _PC)
+_sig("dt_sharded_partials_bytes", _sz, _PC)
+_sig("dt_sharded_build_begin", _i32, _PC, _vp, _vp, _vp, _vp, ctypes.POINTER(DtTree), _vp, _sz, _vp)
+_sig("dt_sharded_build_gemm", _i32, _PC, _i32, _i32, _vp, _i32, _vp, _vp, _vp, _sz, _vp, _vp)
+_sig("dt_sharded_build_frontier", _i32, _PC, _i32, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(DtTree),
+     _vp, _sz, _vp)
 _sig("dt_read_status", _i32, _vp, _vp, ctypes.POINTER(ctypes.c_int32))
 _sig("dt_set_profile_events", None, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int32),
      _i32, ctypes.POINTER(ctypes.c_int32))

@@ -101,10 +101,12 @@ struct BuildLayout {
   int ncta_v, n_vtiles, nt, Mcap, Mcap_pad, Mmat, Mmat_pad;
 };
 
-static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k, int Nmax) {
+// ncta: partials per node (0: one per SM, at most one per vocabulary tile)
+static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k, int Nmax,
+                                int ncta = 0) {
   BuildLayout L;
   L.n_vtiles = (V + 127) / 128;
-  L.ncta_v = std::min(num_sms(), L.n_vtiles);
+  L.ncta_v = ncta > 0 ? ncta : std::min(num_sms(), L.n_vtiles);
   L.nt = gemm_node_tile(Nmax);
   L.Mcap = batch * Nmax;
   L.Mcap_pad = (int)align_up(L.Mcap, L.nt);
@@ -166,6 +168,81 @@ __global__ void chain_cond_kernel(dt_tree chain, const int32_t* root, int batch,
   }
 }
 
+
+// Frontier arguments of a build laid out by L.
+static FrontierArgs frontier_args(const BuildLayout& L, const uint16_t* d_markov_a,
+                                  const float* d_calib, const int32_t* d_n_budget,
+                                  const int32_t* d_k_req, const float* d_lambda, int batch,
+                                  int Bk, int V, int r, int k, int Nmax, float temp,
+                                  const dt_tree* out) {
+  FrontierArgs f;
+  memset(&f, 0, sizeof(f));
+  f.mat_rows = L.mat_rows;
+  f.mat_count = L.counts + 2;
+  // the GEMM gathers its node rows A[token] itself when they fit in shared
+  // memory; otherwise the frontier writes them to H / Hm for TMA
+  const bool gather = gemm_can_gather(r, L.nt);
+  f.H = gather ? nullptr : L.H;
+  f.Hm = gather ? nullptr : L.Hm;
+  f.A = d_markov_a;
+  f.req = L.req;
+  f.lists = L.lists;
+  f.pstats = L.pstats;
+  f.plv = L.plv;
+  f.pli = L.pli;
+  f.pgv = L.pgv;
+  f.pgi = L.pgi;
+  f.ncta = L.ncta_v;
+  f.calib = d_calib;
+  f.n_budget = d_n_budget;
+  f.k_req = d_k_req;
+  f.lambda = d_lambda;
+  f.Mcap = L.Mcap;
+  f.Bk = Bk;
+  f.V = V;
+  f.r = r;
+  f.k = k;
+  f.Nmax = Nmax;
+  f.batch = batch;
+  f.temp = temp;
+  f.out = *out;
+  f.status = L.status;
+  return f;
+}
+
+// Expansion-GEMM arguments of a build laid out by L (the whole vocabulary).
+static GemmArgs gemm_args(const BuildLayout& L, const void* d_block_logits, dt_dtype ldt,
+                          const uint16_t* d_markov_a, int batch, int Bk, int V, int r, int k,
+                          int Nmax, float temp, uint64_t philox_seed, uint64_t philox_offset) {
+  (void)batch;
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.L = d_block_logits;
+  g.l_bf16 = ldt == DT_BF16;
+  g.gatherA = gemm_can_gather(r, L.nt) ? d_markov_a : nullptr;
+  g.Bk = Bk;
+  g.V = V;
+  g.vfull = V;
+  g.r = r;
+  g.k = k;
+  g.n_vtiles = L.n_vtiles;
+  g.ncta_v = L.ncta_v;
+  g.Mcap = L.Mcap;
+  g.temp = temp;
+  g.seed = philox_seed;
+  g.offset = (uint32_t)philox_offset;
+  g.pstats = L.pstats;
+  g.plv = L.plv;
+  g.pli = L.pli;
+  g.pgv = L.pgv;
+  g.pgi = L.pgi;
+  g.nmax1 = Nmax + 1;
+  g.status = L.status;
+  // a wave's column count is only known on the device: one CTA per weight
+  // range loops over the node tiles that have columns
+  g.n_nslots = 1;
+  return g;
+}
 
 // init + Bk waves of GEMM and frontier (+ the draft-q pass at T > 0)
 static dt_status run_waves(FrontierArgs f, GemmArgs g, const BuildLayout& L,
@@ -302,64 +379,10 @@ static dt_status build_impl(const void* d_block_logits, dt_dtype ldt, const uint
 
   if (cudaMemsetAsync(L.status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
 
-  FrontierArgs f;
-  memset(&f, 0, sizeof(f));
-  f.mat_rows = L.mat_rows;
-  f.mat_count = L.counts + 2;
-  // the GEMM gathers its node rows A[token] itself when they fit in shared
-  // memory; otherwise the frontier writes them to H / Hm for TMA
-  const bool gather = gemm_can_gather(r, L.nt);
-  f.H = gather ? nullptr : L.H;
-  f.Hm = gather ? nullptr : L.Hm;
-  f.A = d_markov_a;
-  f.req = L.req;
-  f.lists = L.lists;
-  f.pstats = L.pstats;
-  f.plv = L.plv;
-  f.pli = L.pli;
-  f.pgv = L.pgv;
-  f.pgi = L.pgi;
-  f.ncta = L.ncta_v;
-  f.calib = d_calib;
-  f.n_budget = d_n_budget;
-  f.k_req = d_k_req;
-  f.lambda = d_lambda;
-  f.Mcap = L.Mcap;
-  f.Bk = Bk;
-  f.V = V;
-  f.r = r;
-  f.k = k;
-  f.Nmax = Nmax;
-  f.batch = batch;
-  f.temp = temp;
-  f.out = *out;
-  f.status = L.status;
-
-  GemmArgs g;
-  memset(&g, 0, sizeof(g));
-  g.L = d_block_logits;
-  g.l_bf16 = ldt == DT_BF16;
-  g.gatherA = gather ? d_markov_a : nullptr;
-  g.Bk = Bk;
-  g.V = V;
-  g.r = r;
-  g.k = k;
-  g.n_vtiles = L.n_vtiles;
-  g.ncta_v = L.ncta_v;
-  g.Mcap = L.Mcap;
-  g.temp = temp;
-  g.seed = philox_seed;
-  g.offset = (uint32_t)philox_offset;
-  g.pstats = L.pstats;
-  g.plv = L.plv;
-  g.pli = L.pli;
-  g.pgv = L.pgv;
-  g.pgi = L.pgi;
-  g.nmax1 = Nmax + 1;
-  g.status = L.status;
-  // a wave's column count is only known on the device: one CTA per weight
-  // range loops over the node tiles that have columns
-  g.n_nslots = 1;
+  FrontierArgs f = frontier_args(L, d_markov_a, d_calib, d_n_budget, d_k_req, d_lambda, batch,
+                                 Bk, V, r, k, Nmax, temp, out);
+  GemmArgs g = gemm_args(L, d_block_logits, ldt, d_markov_a, batch, Bk, V, r, k, Nmax, temp,
+                         philox_seed, philox_offset);
 
   if (variant == DT_TREE_CHAIN) {
     // the method with one child per node (k = 1 everywhere)
@@ -399,6 +422,210 @@ static dt_status build_impl(const void* d_block_logits, dt_dtype ldt, const uint
 }
 
 }  // namespace dt
+
+// --------------------------------------------------- vocabulary-sharded build --
+namespace dt {
+
+// Tiles [t_lo, t_hi) of rank `rank` among `world` (the tiles split as evenly
+// as whole tiles allow, lower ranks first).
+static void shard_range(int V, int world, int rank, int* v_base, int* v_len) {
+  const int T = (V + 127) / 128;
+  const int t_lo = (int)((long long)rank * T / world);
+  const int t_hi = (int)((long long)(rank + 1) * T / world);
+  *v_base = t_lo * 128;
+  *v_len = std::min(V, t_hi * 128) - *v_base;
+}
+
+static bool shard_cfg_ok(const dt_shard_cfg* c) {
+  return c && c->batch >= 1 && c->batch <= 1024 && c->Bk >= 1 && c->Bk <= 16 && c->k >= 1 &&
+         c->k <= 16 && c->k <= c->V && c->Nmax >= 1 && c->Nmax <= 64 && c->V >= 1 &&
+         c->V < (1 << 20) && c->r >= 16 && c->r <= 1024 && c->r % 16 == 0 && c->world >= 1 &&
+         c->world <= 64 && c->ncta >= 1 && c->ncta * c->world <= 64 * 148 &&
+         c->ncta <= ((c->V + 127) / 128) / c->world;
+}
+
+// One rank's partials of a wave: statistics [Mcap][ncta], list values and
+// tokens [Mcap][k][ncta].
+struct ShardBlock {
+  float2* pstats;
+  float* plv;
+  int32_t* pli;
+  size_t off_lv, off_li;  // byte offsets of plv and pli within the block
+  size_t bytes;
+};
+
+static ShardBlock shard_block(void* base, const dt_shard_cfg* c) {
+  ShardBlock s;
+  Carver cv{(uint8_t*)base, 0};
+  const size_t np = (size_t)c->batch * c->Nmax * c->ncta;
+  s.pstats = cv.take<float2>(np);
+  s.off_lv = align_up(cv.off, 256);
+  s.plv = cv.take<float>(np * c->k);
+  s.off_li = align_up(cv.off, 256);
+  s.pli = cv.take<int32_t>(np * c->k);
+  s.bytes = align_up(cv.off, 256);
+  return s;
+}
+
+// The gathered blocks [world] -> the frontier's [row][k][world * ncta]
+// layout, for the rows of this wave.
+__global__ void shard_interleave_kernel(const uint8_t* gathered, size_t block_bytes,
+                                        size_t off_lv, size_t off_li, int world, int ncta, int k,
+                                        const int32_t* n_rows, int Mcap, float2* pstats,
+                                        float* plv, int32_t* pli) {
+  const int rows = min(max(*n_rows, 0), Mcap);
+  const int nt = world * ncta;
+  const long long per_row = (long long)nt * (1 + k);
+  const long long total = (long long)rows * per_row;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int row = (int)(e / per_row);
+    const int rem = (int)(e % per_row);
+    const int i = rem / nt - 1;  // -1: statistics, else list entry i
+    const int col = rem % nt;
+    const int w = col / ncta, c = col % ncta;
+    const uint8_t* blk = gathered + (size_t)w * block_bytes;
+    if (i < 0) {
+      pstats[(size_t)row * nt + col] = ((const float2*)blk)[(size_t)row * ncta + c];
+    } else {
+      const size_t src = ((size_t)row * k + i) * ncta + c;
+      const size_t dst = ((size_t)row * k + i) * nt + col;
+      plv[dst] = ((const float*)(blk + off_lv))[src];
+      pli[dst] = ((const int32_t*)(blk + off_li))[src];
+    }
+  }
+}
+
+}  // namespace dt
+
+extern "C" {
+
+void dt_shard_range(int V, int world, int rank, int* v_base, int* v_len) {
+  if (!v_base || !v_len) return;
+  if (V < 1 || world < 1 || rank < 0 || rank >= world) {
+    *v_base = *v_len = 0;
+    return;
+  }
+  shard_range(V, world, rank, v_base, v_len);
+}
+
+int dt_shard_ncta(int V, int world) {
+  if (V < 1 || world < 1) return 0;
+  return std::max(0, std::min(num_sms(), ((V + 127) / 128) / world));
+}
+
+size_t dt_sharded_workspace_bytes(const dt_shard_cfg* c) {
+  if (!shard_cfg_ok(c)) return 0;
+  return build_layout(nullptr, c->batch, c->Bk, c->V, c->r, c->k, c->Nmax, c->world * c->ncta)
+      .bytes;
+}
+
+size_t dt_sharded_partials_bytes(const dt_shard_cfg* c) {
+  if (!shard_cfg_ok(c)) return 0;
+  return shard_block(nullptr, c).bytes;
+}
+
+dt_status dt_sharded_build_begin(const dt_shard_cfg* c, const int32_t* d_root_token,
+                                 const int32_t* d_n_budget, const int32_t* d_k_req,
+                                 const float* d_lambda, const dt_tree* out, void* ws,
+                                 size_t ws_bytes, dt_stream stream) {
+  if (!shard_cfg_ok(c)) return c ? DT_EUNSUPPORTED : DT_EINVAL;
+  if (!d_root_token || !d_n_budget || !d_lambda || !out || !out->d_tokens || !out->d_parents ||
+      !out->d_depths || !out->d_ranks || !out->d_keys || !out->d_anc || !out->d_n_nodes)
+    return DT_EINVAL;
+  BuildLayout L = build_layout(nullptr, c->batch, c->Bk, c->V, c->r, c->k, c->Nmax,
+                               c->world * c->ncta);
+  if (!ws || ws_bytes < L.bytes) return DT_EWORKSPACE;
+  L = build_layout(ws, c->batch, c->Bk, c->V, c->r, c->k, c->Nmax, c->world * c->ncta);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(L.status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
+  FrontierArgs f = frontier_args(L, nullptr, nullptr, d_n_budget, d_k_req, d_lambda, c->batch,
+                                 c->Bk, c->V, c->r, c->k, c->Nmax, 0.f, out);
+  f.H = nullptr;  // the sharded GEMM always gathers its node rows
+  f.Hm = nullptr;
+  ProfileScope ps(DT_K_BUILD_INIT, s);
+  return launch_build_init(f, d_root_token, L.rows[0], L.counts + 0, s) == cudaSuccess
+             ? DT_OK
+             : DT_ECUDA;
+}
+
+dt_status dt_sharded_build_gemm(const dt_shard_cfg* c, int wave, int rank,
+                                const void* d_block_logits, dt_dtype ldt,
+                                const uint16_t* d_markov_a, const uint16_t* d_markov_b_shard,
+                                void* ws, size_t ws_bytes, void* d_partials,
+                                dt_stream stream) {
+  if (!shard_cfg_ok(c)) return c ? DT_EUNSUPPORTED : DT_EINVAL;
+  if (!d_block_logits || !d_markov_a || !d_markov_b_shard || !d_partials) return DT_EINVAL;
+  if (ldt != DT_F32 && ldt != DT_BF16) return DT_EINVAL;
+  if (wave < 0 || wave >= c->Bk || rank < 0 || rank >= c->world) return DT_EINVAL;
+  if ((uintptr_t)d_partials % 256) return DT_EINVAL;
+  BuildLayout L = build_layout(nullptr, c->batch, c->Bk, c->V, c->r, c->k, c->Nmax,
+                               c->world * c->ncta);
+  if (!ws || ws_bytes < L.bytes) return DT_EWORKSPACE;
+  if (!gemm_can_gather(c->r, L.nt)) return DT_EUNSUPPORTED;
+  L = build_layout(ws, c->batch, c->Bk, c->V, c->r, c->k, c->Nmax, c->world * c->ncta);
+  int v_base = 0, v_len = 0;
+  shard_range(c->V, c->world, rank, &v_base, &v_len);
+  CUtensorMap tmW;
+  if (!make_tmap_bf16_kmajor(&tmW, d_markov_b_shard, c->r, v_len, 128)) return DT_ECUDA;
+  const ShardBlock blk = shard_block(d_partials, c);
+  GemmArgs g = gemm_args(L, d_block_logits, ldt, d_markov_a, c->batch, c->Bk, c->V, c->r, c->k,
+                         c->Nmax, 0.f, 0, 0);
+  g.V = v_len;  // this shard's rows of Bm
+  g.v_base = v_base;
+  g.vfull = c->V;
+  g.n_vtiles = (v_len + 127) / 128;
+  g.ncta_v = c->ncta;
+  g.pstats = blk.pstats;
+  g.plv = blk.plv;
+  g.pli = blk.pli;
+  g.pgv = nullptr;
+  g.pgi = nullptr;
+  const int cur = wave & 1;
+  g.rows = L.rows[cur];
+  g.n_rows = L.counts + cur;
+  g.reset_count = L.counts + (cur ^ 1);
+  ProfileScope ps(DT_K_MARKOV_GEMM, (cudaStream_t)stream);
+  return launch_markov_gemm(EPI_EXPAND, false, tmW, tmW, tmW, g, c->batch, L.nt,
+                            (cudaStream_t)stream) == cudaSuccess
+             ? DT_OK
+             : DT_ECUDA;
+}
+
+dt_status dt_sharded_build_frontier(const dt_shard_cfg* c, int wave, const void* d_gathered,
+                                    const float* d_calib, const int32_t* d_n_budget,
+                                    const int32_t* d_k_req, const float* d_lambda,
+                                    const dt_tree* out, void* ws, size_t ws_bytes,
+                                    dt_stream stream) {
+  if (!shard_cfg_ok(c)) return c ? DT_EUNSUPPORTED : DT_EINVAL;
+  if (!d_gathered || !d_n_budget || !d_lambda || !out) return DT_EINVAL;
+  if (wave < 0 || wave >= c->Bk) return DT_EINVAL;
+  BuildLayout L = build_layout(nullptr, c->batch, c->Bk, c->V, c->r, c->k, c->Nmax,
+                               c->world * c->ncta);
+  if (!ws || ws_bytes < L.bytes) return DT_EWORKSPACE;
+  L = build_layout(ws, c->batch, c->Bk, c->V, c->r, c->k, c->Nmax, c->world * c->ncta);
+  cudaStream_t s = (cudaStream_t)stream;
+  const ShardBlock rel = shard_block(nullptr, c);  // layout of one rank's block
+  const int cur = wave & 1;
+  {
+    ProfileScope ps(DT_K_OTHER, s);
+    shard_interleave_kernel<<<num_sms(), 256, 0, s>>>(
+        (const uint8_t*)d_gathered, rel.bytes, rel.off_lv, rel.off_li, c->world, c->ncta, c->k,
+        L.counts + cur, L.Mcap, L.pstats, L.plv, L.pli);
+    if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+  }
+  FrontierArgs f = frontier_args(L, nullptr, d_calib, d_n_budget, d_k_req, d_lambda, c->batch,
+                                 c->Bk, c->V, c->r, c->k, c->Nmax, 0.f, out);
+  f.H = nullptr;
+  f.Hm = nullptr;
+  f.rows = L.rows[cur];
+  f.next_rows = L.rows[cur ^ 1];
+  f.next_count = L.counts + (cur ^ 1);
+  ProfileScope ps(DT_K_FRONTIER, s);
+  return launch_frontier(f, s) == cudaSuccess ? DT_OK : DT_ECUDA;
+}
+
+}  // extern "C"
 
 extern "C" {
 

@@ -52,6 +52,8 @@ struct GemmArgs {
   const void* L;         // bias rows [batch][Bk][V] (block logits, residual) or NULL
   int l_bf16;
   int Bk, V, r, k;       // V: weight rows (vocabulary / features), r: inner dimension
+  int vfull;             // vocabulary of the block logits and of A (0: V); V < vfull for a shard
+  int v_base;            // first token of this launch's vocabulary shard (EXPAND only)
   const Row* rows;       // GEMM columns
   const int32_t* n_rows; // device count of valid columns
   int32_t* reset_count;  // set to 0 by CTA (0,0) (next wave's counter), may be NULL

@@ -374,14 +374,15 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
           } else {
             cm.valid = 1;
             cm.b = r.b;
-            cm.bias_off = ((int64_t)r.b * a.Bk + r.depth) * a.V;
+            // block-logit row over the full vocabulary, from this shard's first token
+            cm.bias_off = ((int64_t)r.b * a.Bk + r.depth) * a.vfull + a.v_base;
             cm.c1 = (uint32_t)r.path;
             cm.c2 = (uint32_t)(r.path >> 32);
             cm.lse = r.lse;
             cm.out_row = r.aux;
             cm.token = r.token;
             // token -1: no Markov term (zero row); anything else must index A
-            if (gather && (r.token < -1 || r.token >= a.V)) {
+            if (gather && (r.token < -1 || r.token >= a.vfull)) {
               set_status(a.status, DT_EDEVICE);
               cm.valid = 0;
             }
@@ -700,7 +701,8 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
         named_bar(1, S::kEpiWarps * 32);
       }
       const bool ldg_bias = S::CPT == 1 && a.L != nullptr && !cached;
-      const bool vec = (a.l_bf16 ? (a.V % 8 == 0) : (a.V % 4 == 0)) && ((uintptr_t)a.L % 16 == 0);
+      const bool vec = (a.l_bf16 ? (a.vfull % 8 == 0) : (a.vfull % 4 == 0)) &&
+                       ((uintptr_t)a.L % 16 == 0);
       uint4 raw[8];
       bool raw_ok = false;
       if (ldg_bias) {
@@ -806,7 +808,7 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
   #pragma unroll
             for (int i = 0; i < 32; ++i) {
               if (s[i] > thr[j]) {
-                topk_insert<KMAX>(L1[j], I1[j], s[i], xq + i);
+                topk_insert<KMAX>(L1[j], I1[j], s[i], a.v_base + xq + i);
                 thr[j] = kth<KMAX>(L1[j], k);
               }
             }
@@ -819,7 +821,7 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
                 const float smax =
                     fmaxf(fmaxf(s[4 * gi], s[4 * gi + 1]), fmaxf(s[4 * gi + 2], s[4 * gi + 3]));
                 if (!(smax + kGumbelMax > gthr[j])) continue;
-                const uint32_t x4 = (uint32_t)(xq + 4 * gi);
+                const uint32_t x4 = (uint32_t)(a.v_base + xq + 4 * gi);
                 const U4 o = philox10(
                     U4{(x4 >> 2) | ((uint32_t)mc[j].b << 18), mc[j].c1, mc[j].c2, a.offset},
                     (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
@@ -830,7 +832,7 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
                   if (i >= nv) continue;
                   const float gk = s[i] + (-logf(-logf(u23(wds[jj]))));
                   if (gk > gthr[j]) {
-                    topk_insert<KMAX>(L2[j], I2[j], gk, xq + i);
+                    topk_insert<KMAX>(L2[j], I2[j], gk, a.v_base + xq + i);
                     gthr[j] = kth<KMAX>(L2[j], k);
                   }
                 }
@@ -983,7 +985,7 @@ static cudaError_t launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmW2,
   a.bias_rows = 0;
   if (MODE != EPI_SWIGLU && a.L) {
     const int esz = a.l_bf16 ? 2 : 4;
-    const bool aligned = ((uintptr_t)a.L % 16 == 0) && ((size_t)a.V * esz) % 16 == 0;
+    const bool aligned = ((uintptr_t)a.L % 16 == 0) && ((size_t)a.vfull * esz) % 16 == 0;
     const int span = ((a.n_vtiles + a.ncta_v - 1) / a.ncta_v) * 128;
     // distinct rows a node tile can need: one per (request, depth), at most NT
     const int rows = std::min(std::min(SH::NT, kBiasRowsMax), batch * a.Bk);
@@ -1030,6 +1032,9 @@ cudaError_t launch_markov_gemm(int mode, bool stoch, const CUtensorMap& tmW,
                                int batch, int nt, cudaStream_t s) {
   const int ng = nt / 32;
   a.n_ntiles = (a.Mcap + nt - 1) / nt;
+  if (a.vfull == 0) a.vfull = a.V;
+  // a vocabulary shard starts on a tile and only expands nodes
+  if (a.v_base != 0 && (mode != EPI_EXPAND || a.v_base % kTileV)) return cudaErrorInvalidValue;
   // node-tile slots per weight range: every tile gets its own CTA unless the
   // caller asks for fewer (then each CTA loops over tiles)
   a.n_nslots = (a.n_nslots > 0 && a.n_nslots < a.n_ntiles) ? a.n_nslots : a.n_ntiles;

@@ -9,6 +9,8 @@
  *   dt_tree_load_budget cut a batch of trees to a round's verification
  *                       capacity by survival (load-adaptive tree size)
  *   dt_calib_log/_fit   log verified rounds and fit the calibration
+ *   dt_sharded_build_*  the build with the Markov factor split by vocabulary
+ *                       over several GPUs (partials all-gathered per wave)
  *   dt_tree_verify_attn tree-masked grouped-query attention over prefix + tree
  *   dt_tree_accept      lossless acceptance walk (greedy or recursive residual)
  *
@@ -281,6 +283,63 @@ dt_status dt_tree_accept_noalloc(const void* d_target_logits, dt_dtype tdt,
                                  uint64_t philox_offset, int32_t* d_acc_nodes,
                                  int32_t* d_n_acc, int32_t* d_bonus,
                                  dt_stream stream);
+
+/* ---------------------------------------------- vocabulary-sharded build --
+ * dt_tree_build (T = 0) with the Markov factor Bm split by vocabulary over
+ * `world` ranks (one process per GPU), for a Bm too large for one GPU or to
+ * spread one request's weight stream over several GPUs.  Rank w holds the
+ * rows [v_base, v_base + v_len) of Bm given by dt_shard_range (whole
+ * 128-token tiles, split as evenly as tiles allow); every rank holds the
+ * block logits, A and the request arrays, and builds the same tree.  Per
+ * wave w = 0 .. Bk-1 the caller runs, on every rank:
+ *   dt_sharded_build_gemm      this rank's expansion GEMM over its shard:
+ *                              per node row, `ncta` partial (max, sum exp)
+ *                              statistics and top-k lists, into d_partials
+ *                              (dt_sharded_partials_bytes, 256-byte aligned);
+ *   an all-gather of the partial blocks in rank order (e.g. NCCL), giving
+ *                              [world][block] at d_gathered;
+ *   dt_sharded_build_frontier  merges the world * ncta partials per node
+ *                              (log-sum-exp and the k best, exactly as the
+ *                              one-GPU build merges its per-CTA partials)
+ *                              and runs the best-first frontier.
+ * after dt_sharded_build_begin, which clears the status word and seeds wave 0
+ * with the roots.  Every rank takes the same decisions from the same merged
+ * values, so the trees are identical; each equals dt_tree_build's on the
+ * same inputs up to the fp32 order of the log-sum-exp (keys within 1e-5).
+ *   cfg.ncta   partials per rank: dt_shard_ncta(V, world) (one per SM, at
+ *              most the smallest shard's tile count), the same on all ranks
+ *   limits     those of dt_tree_build with r <= 512 (Nmax <= 32) or r <= 256
+ *              (Nmax <= 64), so that the GEMM gathers its node rows in shared
+ *              memory; world <= 64
+ *   ws         >= dt_sharded_workspace_bytes(&cfg), one per rank
+ * Device-side checks report through the status word of ws. */
+typedef struct {
+  int batch, Bk, V, r, k, Nmax; /* as dt_tree_build (V: the whole vocabulary) */
+  int world;                    /* ranks sharing the vocabulary */
+  int ncta;                     /* partials per rank per node row */
+} dt_shard_cfg;
+
+void dt_shard_range(int V, int world, int rank, int* v_base, int* v_len);
+int dt_shard_ncta(int V, int world);
+size_t dt_sharded_workspace_bytes(const dt_shard_cfg* cfg);
+size_t dt_sharded_partials_bytes(const dt_shard_cfg* cfg);
+
+dt_status dt_sharded_build_begin(const dt_shard_cfg* cfg, const int32_t* d_root_token,
+                                 const int32_t* d_n_budget, const int32_t* d_k_req,
+                                 const float* d_lambda, const dt_tree* out, void* ws,
+                                 size_t ws_bytes, dt_stream stream);
+
+dt_status dt_sharded_build_gemm(const dt_shard_cfg* cfg, int wave, int rank,
+                                const void* d_block_logits, dt_dtype ldt,
+                                const uint16_t* d_markov_a,
+                                const uint16_t* d_markov_b_shard, void* ws,
+                                size_t ws_bytes, void* d_partials, dt_stream stream);
+
+dt_status dt_sharded_build_frontier(const dt_shard_cfg* cfg, int wave, const void* d_gathered,
+                                    const float* d_calib, const int32_t* d_n_budget,
+                                    const int32_t* d_k_req, const float* d_lambda,
+                                    const dt_tree* out, void* ws, size_t ws_bytes,
+                                    dt_stream stream);
 
 /* ---------------------------------------------------------- load policy --
  * Load-adaptive tree size (TreeSpark article, "core idea": the load-adaptive
