@@ -99,6 +99,7 @@ struct BuildLayout {
   float* chain_lam;    // [batch] Shared-Markov chain: no survival stop
   size_t bytes;
   int ncta_v, n_vtiles, nt, Mcap, Mcap_pad, Mmat, Mmat_pad;
+  int nt_x;  // node tile of the expansion GEMMs
 };
 
 // ncta: partials per node (0: one per SM, at most one per vocabulary tile)
@@ -108,6 +109,10 @@ static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k
   L.n_vtiles = (V + 127) / 128;
   L.ncta_v = ncta > 0 ? ncta : std::min(num_sms(), L.n_vtiles);
   L.nt = gemm_node_tile(Nmax);
+  // With several requests a wave has many columns: 64-column tiles halve the
+  // passes over the weights and give the epilogue two warps per quadrant
+  // (when the rows still fit the shared-memory gather).
+  L.nt_x = (batch > 1 && L.nt == 32 && gemm_can_gather(r, 64)) ? 64 : L.nt;
   L.Mcap = batch * Nmax;
   L.Mcap_pad = (int)align_up(L.Mcap, L.nt);
   L.Mmat = batch * (Nmax + 1);
@@ -262,7 +267,8 @@ static dt_status run_waves(FrontierArgs f, GemmArgs g, const BuildLayout& L,
     g.reset_count = L.counts + nxt;
     {
       ProfileScope ps(DT_K_MARKOV_GEMM, s);
-      if (launch_markov_gemm(EPI_EXPAND, stoch, tmW, tmW, tmH, g, batch, L.nt, s) != cudaSuccess)
+      if (launch_markov_gemm(EPI_EXPAND, stoch, tmW, tmW, tmH, g, batch, L.nt_x, s) !=
+          cudaSuccess)
         return DT_ECUDA;
     }
     f.rows = L.rows[cur];
@@ -562,7 +568,7 @@ dt_status dt_sharded_build_gemm(const dt_shard_cfg* c, int wave, int rank,
   BuildLayout L = build_layout(nullptr, c->batch, c->Bk, c->V, c->r, c->k, c->Nmax,
                                c->world * c->ncta);
   if (!ws || ws_bytes < L.bytes) return DT_EWORKSPACE;
-  if (!gemm_can_gather(c->r, L.nt)) return DT_EUNSUPPORTED;
+  if (!gemm_can_gather(c->r, L.nt_x)) return DT_EUNSUPPORTED;
   L = build_layout(ws, c->batch, c->Bk, c->V, c->r, c->k, c->Nmax, c->world * c->ncta);
   int v_base = 0, v_len = 0;
   shard_range(c->V, c->world, rank, &v_base, &v_len);
@@ -586,7 +592,7 @@ dt_status dt_sharded_build_gemm(const dt_shard_cfg* c, int wave, int rank,
   g.n_rows = L.counts + cur;
   g.reset_count = L.counts + (cur ^ 1);
   ProfileScope ps(DT_K_MARKOV_GEMM, (cudaStream_t)stream);
-  return launch_markov_gemm(EPI_EXPAND, false, tmW, tmW, tmW, g, c->batch, L.nt,
+  return launch_markov_gemm(EPI_EXPAND, false, tmW, tmW, tmW, g, c->batch, L.nt_x,
                             (cudaStream_t)stream) == cudaSuccess
              ? DT_OK
              : DT_ECUDA;
