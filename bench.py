@@ -400,12 +400,26 @@ def run_ours(args):
     d2h = sum(t.numel() * t.element_size() for t in h_out.values())
     c = copies[0]
     ke = min(args.steps, 50)
+    # the target rows are only read by the accept walk: their copy runs on a
+    # second stream beside the build and the verify attention
+    side = torch.cuda.Stream(device=dev)
+    tgt_ready, tgt_free = torch.cuda.Event(), torch.cuda.Event()
+    tgt_free.record(stream)
     with torch.cuda.stream(stream):
         def e2e_step():
+            side.wait_event(tgt_free)          # the previous walk has read its rows
+            with torch.cuda.stream(side):
+                c["tgt"].copy_(h_in["tgt"], non_blocking=True)
+                tgt_ready.record(side)
             for nm, t in h_in.items():
-                c[nm].copy_(t, non_blocking=True)
+                if nm != "tgt":
+                    c[nm].copy_(t, non_blocking=True)
             c["root"].copy_(h_root, non_blocking=True)
-            round_(c)
+            build(c)
+            verify(c)
+            stream.wait_event(tgt_ready)
+            accept_(c)
+            tgt_free.record(stream)
             h_out["tok"].copy_(tree.tokens, non_blocking=True)
             h_out["par"].copy_(tree.parents, non_blocking=True)
             h_out["n"].copy_(tree.n_nodes, non_blocking=True)
@@ -418,15 +432,17 @@ def run_ours(args):
         barrier()
         e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e2.record(stream)
+        side.wait_event(e2)  # no side-stream copy starts before the timed region
         for _ in range(ke):
             e2e_step()
-        e3.record(stream)
+        e3.record(stream)    # after the last walk, which waited for the last copy
     torch.cuda.synchronize()
     barrier()
     ms_e = max_over_ranks(e2.elapsed_time(e3), world, dev)
     e2e = {"value": round(job_throughput(ke, world, ms_e), 1), "unit": UNIT,
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": ke,
-           "path": "python API (eager launches) + pinned H2D/D2H copies on the stream"}
+           "path": "python API (eager launches) + pinned H2D/D2H copies; the target rows "
+                   "are copied on a second stream beside build and verify"}
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
