@@ -77,3 +77,39 @@ def test_accept_and_attention_reject_bad_arguments():
                                      None, 0, None) == L.DT_EUNSUPPORTED
     assert L.lib.dt_tree_verify_attn(p, p, p, p, p, 32, p, p, p, p, 1, 8, 6, 4, 64, 0.1, 1, p,
                                      None, 0, None) == L.DT_EINVAL
+
+
+def test_new_entry_points_reject_bad_arguments_without_a_device():
+    import draft_tree_construction_markov_b200._lib as L
+    p = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+    tree = L.DtTree(p, p, p, p, p, p, p, p)
+    t = ctypes.byref(tree)
+    # baseline variants: an unknown variant
+    assert L.lib.dt_tree_build_ex(p, 1, p, p, 16, None, p, p, None, p, 1, 4, 512, 2, 8, 0.0, 0, 0,
+                                  7, t, p, 1 << 20, None) == L.DT_EINVAL
+    # load budget: negative capacity, too large a batch, no workspace
+    assert L.lib.dt_tree_load_budget(t, 2, 8, None, -1, 0, None, p, 256, None) == L.DT_EINVAL
+    assert L.lib.dt_tree_load_budget(t, 1025, 8, None, 5, 0, None, p, 256, None) == \
+        L.DT_EUNSUPPORTED
+    assert L.lib.dt_tree_load_budget(t, 2, 8, None, 5, 0, None, None, 0, None) == L.DT_EWORKSPACE
+    # calibration: negative alpha start, too large a grid, too small a workspace
+    assert L.lib.dt_calib_fit(p, p, p, 10, 4, -1.0, 0.1, 4, 0.0, 0.1, 4, 1, p, None, p, 4096,
+                              None) == L.DT_EINVAL
+    assert L.lib.dt_calib_fit(p, p, p, 10, 4, 0.0, 0.1, 2048, 0.0, 0.1, 1024, 1, p, None, p,
+                              1 << 30, None) == L.DT_EUNSUPPORTED
+    need = L.lib.dt_calib_workspace_bytes(4, 64, 64)
+    assert need > 256
+    assert L.lib.dt_calib_fit(p, p, p, 10, 4, 0.0, 0.1, 64, 0.0, 0.1, 64, 1, p, None, p, need - 1,
+                              None) == L.DT_EWORKSPACE
+    assert L.lib.dt_calib_log(t, p, p, 1025, 4, 8, p, p, p, p, 256, None) == L.DT_EUNSUPPORTED
+    # sharded build: more partials per rank than the smallest shard has tiles
+    bad = L.ShardCfg(1, 4, 512, 16, 2, 8, 2, 3)
+    assert L.lib.dt_sharded_workspace_bytes(ctypes.byref(bad)) == 0
+    assert L.lib.dt_sharded_build_begin(ctypes.byref(bad), p, p, None, p, t, p, 1 << 20,
+                                        None) == L.DT_EUNSUPPORTED
+    good = L.ShardCfg(1, 4, 512, 16, 2, 8, 2, 2)
+    assert L.lib.dt_sharded_workspace_bytes(ctypes.byref(good)) > 0
+    assert L.lib.dt_sharded_build_gemm(ctypes.byref(good), 0, 2, p, 1, p, p, p, 1 << 20, p,
+                                       None) == L.DT_EINVAL      # rank outside the world
+    assert L.lib.dt_sharded_build_frontier(ctypes.byref(good), 4, p, None, p, None, p, t, p,
+                                           1 << 20, None) == L.DT_EINVAL   # wave >= Bk
