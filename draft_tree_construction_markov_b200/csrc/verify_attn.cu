@@ -318,15 +318,32 @@ __global__ void attn_combine_kernel(AttnArgs a) {
   const int nvec = a.d / 4;  // 16 or 32 float4 per row
   if (lane < nvec) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int s = 0; s < used; ++s) {
-      const float2 ml = a.part_ml[pb0 + s * split_stride];
-      const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - mx);
-      const float4 o = ((const float4*)(a.part_o + (pb0 + s * split_stride) * a.d))[lane];
-      acc.x += w * o.x;
-      acc.y += w * o.y;
-      acc.z += w * o.z;
-      acc.w += w * o.w;
+    // kBatch splits per pass: all their loads are issued before the first
+    // use, so a pass costs one memory round trip; the sum keeps split order
+    constexpr int kBatch = 16;
+    for (int s0 = 0; s0 < used; s0 += kBatch) {
+      float2 ml[kBatch];
+      float4 o[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int s = s0 + j;
+        if (s < used) {
+          ml[j] = a.part_ml[pb0 + s * split_stride];
+          o[j] = ((const float4*)(a.part_o + (pb0 + s * split_stride) * a.d))[lane];
+        } else {
+          ml[j] = make_float2(-INFINITY, 0.f);
+          o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        if (s0 + j >= used) break;
+        const float w = ml[j].x == -INFINITY ? 0.f : exp2f(ml[j].x - mx);
+        acc.x += w * o[j].x;
+        acc.y += w * o[j].y;
+        acc.z += w * o[j].z;
+        acc.w += w * o[j].w;
+      }
     }
     const size_t oi = (((size_t)b * (a.Nmax + 1) + i) * a.Hq + h) * a.d + 4 * lane;
     if (a.out_bf16) {
