@@ -21,6 +21,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -142,7 +143,8 @@ class ClockSampler:
         vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
         self.index = vis[local].strip() if local < len(vis) else str(local)
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{local}.csv")
+        # raw samples go to a scratch file; the JSON line carries their summary
+        self.path = os.path.join(tempfile.gettempdir(), f"dtree_clocks_{os.getpid()}_{local}.csv")
 
     def start(self):
         try:
