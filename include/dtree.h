@@ -246,7 +246,10 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix,
  *   d_target_logits [batch][Nmax+1][V] fp32 or bf16, row 0 = root, row i+1 =
  *   node i; tree = the dt_tree of dt_tree_build (d_draft_q needed iff T > 0).
  * Outputs (device): d_acc_nodes [batch][Bk] accepted node indices by depth
- * (-1 padded), d_n_acc [batch], d_bonus [batch]. */
+ * (-1 padded), d_n_acc [batch], d_bonus [batch].
+ * At T > 0 each request's walk runs on one thread-block cluster of up to 8
+ * CTAs of 1024 threads (fewer when the batch would not fit the SMs at once);
+ * a launch that cannot place its clusters returns DT_ECUDA. */
 size_t dt_tree_accept_workspace_bytes(int batch, int Nmax, int V);
 
 dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt,
