@@ -113,3 +113,51 @@ def test_new_entry_points_reject_bad_arguments_without_a_device():
                                        None) == L.DT_EINVAL      # rank outside the world
     assert L.lib.dt_sharded_build_frontier(ctypes.byref(good), 4, p, None, p, None, p, t, p,
                                            1 << 20, None) == L.DT_EINVAL   # wave >= Bk
+
+
+def _prototypes():
+    """name -> [C parameter types] for every function declared in the header."""
+    src = open(os.path.join(ROOT, "include", "dtree.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(dt_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", src):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        types = []
+        for p in params:
+            p = re.sub(r"\s+", " ", p)
+            name = re.search(r"(\w+)\s*$", p).group(1)
+            types.append(p[: p.rfind(name)].strip())
+        out[m.group(1)] = types
+    return out
+
+
+def _ctype_for(c):
+    import ctypes as C
+    if "*" in c:
+        return "ptr"
+    base = c.replace("const ", "").strip()
+    return {"int": C.c_int, "float": C.c_float, "uint64_t": C.c_uint64, "int64_t": C.c_int64,
+            "size_t": C.c_size_t, "dt_dtype": C.c_int, "dt_tree_variant": C.c_int,
+            "dt_stream": "ptr"}[base]
+
+
+def test_binding_signatures_match_the_header():
+    """Every function the binding gives argtypes to has the header's parameter
+    count, and each parameter the same kind (pointer, or the same scalar)."""
+    import ctypes as C
+    import draft_tree_construction_markov_b200._lib as L
+    protos = _prototypes()
+    checked = 0
+    for name, types in protos.items():
+        fn = getattr(L.lib, name)
+        if fn.argtypes is None:
+            continue
+        assert len(fn.argtypes) == len(types), name
+        for i, (ct, at) in enumerate(zip(types, fn.argtypes)):
+            want = _ctype_for(ct)
+            if want == "ptr":
+                assert at is C.c_void_p or issubclass(at, C._Pointer), (name, i, ct, at)
+            else:
+                assert at is want, (name, i, ct, at)
+        checked += 1
+    assert checked >= 20
