@@ -18,6 +18,7 @@ __all__ = ["Tree", "tree_build", "tree_verify_attn", "tree_accept", "markov_logi
            "read_status", "build_workspace_bytes", "verify_workspace_bytes",
            "accept_workspace_bytes", "workspace", "DtreeError", "num_sms", "tree_load_budget",
            "load_budget_workspace_bytes", "calib_workspace_bytes", "calib_log", "calib_fit",
+           "tree_accept_noalloc",
            "shard_range", "shard_cfg", "sharded_workspace_bytes", "sharded_partials_bytes",
            "sharded_build_begin", "sharded_build_gemm", "sharded_build_frontier",
            "tree_build_sharded"]
@@ -129,6 +130,20 @@ def tree_accept(target_logits, tree: Tree, Bk, temp, acc_nodes, n_acc, bonus, ws
         ptr(target_logits), dtype_code(target_logits), ctypes.byref(st), batch, Bk, V, n1 - 1,
         float(temp), philox_seed, philox_offset, ptr(acc_nodes), ptr(n_acc), ptr(bonus), ptr(ws),
         ws.numel(), stream_ptr(stream)), "dt_tree_accept")
+    return acc_nodes, n_acc, bonus
+
+
+def tree_accept_noalloc(target_logits, tree: Tree, Bk, temp, acc_nodes, n_acc, bonus,
+                        philox_seed=0, philox_offset=0, stream=None):
+    """dt_tree_accept_noalloc: dt_tree_accept with the library's fixed scratch
+    (no workspace; batch 1 at V = 151936 fits, larger sizes raise
+    DT_EUNSUPPORTED)."""
+    batch, n1, V = target_logits.shape
+    st = tree.c_struct()
+    check(_lib.lib.dt_tree_accept_noalloc(
+        ptr(target_logits), dtype_code(target_logits), ctypes.byref(st), batch, Bk, V, n1 - 1,
+        float(temp), philox_seed, philox_offset, ptr(acc_nodes), ptr(n_acc), ptr(bonus),
+        stream_ptr(stream)), "dt_tree_accept_noalloc")
     return acc_nodes, n_acc, bonus
 
 

@@ -60,6 +60,8 @@ _sig("dt_tree_verify_attn", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, 
 _sig("dt_tree_accept_workspace_bytes", _sz, _i32, _i32, _i32)
 _sig("dt_tree_accept", _i32, _vp, _i32, ctypes.POINTER(DtTree), _i32, _i32, _i32, _i32, _f32,
      _u64, _u64, _vp, _vp, _vp, _vp, _sz, _vp)
+_sig("dt_tree_accept_noalloc", _i32, _vp, _i32, ctypes.POINTER(DtTree), _i32, _i32, _i32, _i32,
+     _f32, _u64, _u64, _vp, _vp, _vp, _vp)
 _sig("dt_treeflash_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("dt_treeflash_build", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
      _i32, _i32, _i32, _i32, ctypes.POINTER(DtTree), _vp, _sz, _vp)
