@@ -146,6 +146,12 @@ class ClockSampler:
         # raw samples go to a scratch file; the JSON line carries their summary
         self.path = os.path.join(tempfile.gettempdir(), f"dtree_clocks_{os.getpid()}_{local}.csv")
 
+    # nvidia-smi needs a moment before its first sample: the sampler starts
+    # this long before the timed region (outside it), and runs one sampling
+    # interval past its end, so that even a region shorter than the interval
+    # is bracketed by samples
+    LEAD_S, TAIL_S = 1.0, 0.1
+
     def start(self):
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
@@ -155,10 +161,13 @@ class ClockSampler:
                  "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        time.sleep(self.LEAD_S)
 
     def stop(self):
         if self.proc is None:
             return None
+        time.sleep(self.TAIL_S)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)

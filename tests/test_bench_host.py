@@ -1,0 +1,44 @@
+"""Host helpers of bench.py that need no GPU.
+
+The clock sampler is driven by a stand-in `nvidia-smi` on PATH that prints a
+sample every 50 ms: a timed region much shorter than the sampling interval
+must still come back with samples and the throttle reasons they report.
+"""
+import os
+import stat
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+FAKE = """#!{py}
+import time
+while True:
+    print("0, 1965, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Active", flush=True)
+    time.sleep(0.05)
+"""
+
+
+def test_clock_sampler_brackets_a_short_region(tmp_path, monkeypatch):
+    exe = tmp_path / "nvidia-smi"
+    exe.write_text(FAKE.format(py=sys.executable))
+    exe.chmod(exe.stat().st_mode | stat.S_IEXEC)
+    monkeypatch.setenv("PATH", f"{tmp_path}{os.pathsep}{os.environ['PATH']}")
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.ClockSampler(0)
+    c.start()
+    time.sleep(0.005)   # the timed region
+    r = c.stop()
+    assert r is not None and r["samples"] >= 2
+    assert r["sm_mhz"] == 1965.0 and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
+    monkeypatch.setenv("PATH", str(tmp_path))   # nothing to run
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.ClockSampler(0)
+    c.start()
+    assert c.stop() is None
