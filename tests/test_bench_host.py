@@ -42,3 +42,21 @@ def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
     c = bench.ClockSampler(0)
     c.start()
     assert c.stop() is None
+
+
+def test_traffic_is_read_only_for_the_profiled_source(tmp_path, monkeypatch):
+    import hashlib
+    sys.path.insert(0, ROOT)
+    import bench
+    src = tmp_path / "kernel.cu"
+    src.write_text("// kernel v1\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    prof = tmp_path / "profiles" / "markov_gemm_qwen3_4b.txt"
+    prof.write_text(f"# summary\nsource_sha256_16: {sha}\ndram_bytes_per_launch: 80091904\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_from_profile(str(src)) == 80091904.0
+    src.write_text("// kernel v2\n")          # the kernel changed since the capture
+    assert bench.traffic_from_profile(str(src)) is None
+    prof.unlink()
+    assert bench.traffic_from_profile(str(src)) is None
