@@ -137,7 +137,8 @@ def time_oracle(w, target, budget_s=20.0, max_rounds=None):
 class ClockSampler:
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,timestamp")
+    INTERVAL_MS = 20
 
     def __init__(self, local):
         vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
@@ -158,13 +159,18 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", str(self.INTERVAL_MS)], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
             return
         time.sleep(self.LEAD_S)
 
-    def stop(self):
+    def stop(self, region=None):
+        """Summary of the samples.  region = (t0, t1), host wall-clock seconds
+        that bracket the timed region (taken before its first launch and after
+        the synchronize that ends it): only samples inside it are summarised;
+        when it is shorter than the sampling interval and holds none, the last
+        sample before it and the first after it stand in (`window` says which)."""
         if self.proc is None:
             return None
         time.sleep(self.TAIL_S)
@@ -174,24 +180,56 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            c = [x.strip() for x in line.split(",")]
-            if len(c) < 9:
-                continue
-            try:
-                sm.append(float(c[1]))
-                mx = max(mx, float(c[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, c[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return summarise_clocks(open(self.path).read().splitlines(), region)
+
+
+def _smi_time(ts):
+    """nvidia-smi's `timestamp` field (local time) -> seconds since the epoch."""
+    import datetime
+    for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+        try:
+            return datetime.datetime.strptime(ts.strip(), fmt).timestamp()
+        except ValueError:
+            pass
+    return None
+
+
+def summarise_clocks(lines, region=None):
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    rows = []
+    for line in lines:
+        c = [x.strip() for x in line.split(",")]
+        if len(c) < 9:
+            continue
+        try:
+            sm, mx = float(c[1]), float(c[2])
+        except ValueError:
+            continue
+        t = _smi_time(c[9]) if len(c) > 9 else None
+        act = {nm for nm, v in zip(names, c[5:9]) if v.lower() == "active"}
+        rows.append((t, sm, mx, act))
+    if not rows:
+        return None
+    window = "all"
+    if region is not None and all(r[0] is not None for r in rows):
+        t0, t1 = region
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        if inside:
+            sel, window = inside, "region"
+        else:
+            before = [r for r in rows if r[0] < t0]
+            after = [r for r in rows if r[0] > t1]
+            sel = before[-1:] + after[:1]
+            window = "bracketing"
+        n_in = len(inside)
+    else:
+        sel, n_in = rows, None
+    reasons = set()
+    for r in sel:
+        reasons |= r[3]
+    return {"sm_mhz": statistics.median([r[1] for r in sel]),
+            "sm_max_mhz": max(r[2] for r in rows), "reasons": sorted(reasons),
+            "samples": len(rows), "samples_in_region": n_in, "window": window}
 
 
 # ------------------------------------------------------------------- GPU ----
@@ -202,9 +240,61 @@ def peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def traffic_from_profile(kernel_src):
+def build_roofline(kern, *, V, r, B, Bk, inner, lbytes):
+    """Roofline object of the tree build, the round's dominant kernel.
+
+    The algorithmic bytes are those of the whole build: the Markov factor Bm
+    [V][r] bf16 once (the waves of one round re-read it from L2), every
+    block-logit row [B][Bk][V], and the gathered node rows A[token] (`inner`
+    expanded nodes, counted from the final trees); the per-node outputs are a
+    few KB.  With the persistent build one launch is the whole build; with one
+    launch pair per wave the GEMM launches of a round (Bk of them) together
+    are, and each is charged Bm once, as if nothing stayed in L2 between them.
+    """
+    pk, pk_kind = peaks()
+    flops = 2.0 * inner * V * r
+    if "pbuild" in kern:
+        nbytes = V * r * 2 + B * Bk * V * lbytes + inner * r * 2
+        us = kern["pbuild"]["avg_us"]
+        name = ("pbuild (every wave of the build in one launch: tcgen05 Markov-head GEMM, fused "
+                "softmax/top-k epilogue, grid barrier, merge and best-first selection)")
+        src, per = "pbuild.cu", "build"
+    else:
+        cols = inner / Bk
+        nbytes = V * r * 2 + B * V * lbytes + cols * r * 2
+        flops = 2.0 * cols * V * r
+        us = kern["markov_gemm"]["avg_us"]
+        name = "markov_gemm (one wave: tcgen05 Markov-head GEMM + fused softmax/top-k epilogue)"
+        src, per = "markov_gemm.cu", "wave"
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    t_tc = flops / (pk["bf16_tflops"] * 1e12)
+    if t_tc > t_hbm:
+        achieved = flops / (us * 1e-6) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        achieved = nbytes / (us * 1e-6) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s"}
+    roof.update({"frac": round(achieved / roof["peak"], 4), "peak_kind": pk_kind,
+                 "kernel": name, "launch_covers": per,
+                 "algorithmic_bytes_per_launch": int(nbytes),
+                 "algorithmic_flops_per_launch": int(flops),
+                 "expanded_nodes_per_build": int(inner),
+                 "traffic": traffic_from_profile(os.path.join(
+                     ROOT, "draft_tree_construction_markov_b200", "csrc", src)),
+                 "avg_launch_us": round(us, 3)})
+    return roof
+
+
+# ncu summary of each kernel source's launch on the headline workload
+PROFILE_OF = {"markov_gemm.cu": "markov_gemm_qwen3_4b.txt", "pbuild.cu": "pbuild_qwen3_4b.txt"}
+
+
+def traffic_from_profile(kernel_src, profile=None):
     """DRAM bytes per launch recorded from an ncu capture, if the kernel is unchanged."""
-    path = os.path.join(ROOT, "profiles", "markov_gemm_qwen3_4b.txt")
+    profile = profile or PROFILE_OF.get(os.path.basename(kernel_src), "")
+    path = os.path.join(ROOT, "profiles", profile)
     try:
         txt = open(path).read()
     except OSError:
@@ -330,14 +420,16 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_reg0 = time.time()
     with torch.cuda.stream(stream):
         e0.record(stream)
         for i in range(args.steps):
             graphs[i % len(graphs)].replay()
         e1.record(stream)
     torch.cuda.synchronize()
+    t_reg1 = time.time()
     barrier()
-    clk = clocks.stop()
+    clk = clocks.stop((t_reg0, t_reg1))
     ms = e0.elapsed_time(e1)
     ms_max = max_over_ranks(ms, world, dev)
     value = job_throughput(args.steps, world, ms_max)
@@ -369,35 +461,8 @@ def run_ours(args):
     kern = {nm: {"launches_per_step": len(v) / kprof, "avg_us": 1e3 * statistics.mean(v),
                  "us_per_step": 1e3 * sum(v) / kprof} for nm, v in per_kind.items()}
 
-    # ---- roofline of the dominant kernel (the Markov GEMM waves).  Per launch
-    # it must stream the whole Markov factor Bm [V][r] bf16 once, read one
-    # block-logit row per request and the gathered node rows; its outputs
-    # (per-CTA softmax statistics and top-k lists) are a few KB.  `cols` =
-    # expanded nodes per wave, counted from the final trees.
-    pk, pk_kind = peaks()
-    cols = inner / Bk
-    lbytes = 2 if w.logit_dtype == "bf16" else 4
-    gemm_bytes = V * r * 2 + B * V * lbytes + cols * r * 2
-    gemm_flops = 2.0 * cols * V * r
-    g_us = kern["markov_gemm"]["avg_us"]
-    t_hbm = gemm_bytes / (pk["hbm_gbs"] * 1e9)
-    t_tc = gemm_flops / (pk["bf16_tflops"] * 1e12)
-    if t_tc > t_hbm:
-        achieved = gemm_flops / (g_us * 1e-6) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
-                "unit": "TFLOP/s"}
-    else:
-        achieved = gemm_bytes / (g_us * 1e-6) / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
-                "unit": "GB/s"}
-    roof.update({"frac": round(achieved / roof["peak"], 4), "peak_kind": pk_kind,
-                 "kernel": "markov_gemm (one wave: tcgen05 Markov-head GEMM + fused softmax/top-k epilogue)",
-                 "algorithmic_bytes_per_launch": int(gemm_bytes),
-                 "algorithmic_flops_per_launch": int(gemm_flops),
-                 "nodes_per_wave": round(cols, 2),
-                 "traffic": traffic_from_profile(os.path.join(
-                     ROOT, "draft_tree_construction_markov_b200", "csrc", "markov_gemm.cu")),
-                 "avg_launch_us": round(g_us, 3)})
+    roof = build_roofline(kern, V=V, r=r, B=B, Bk=Bk, inner=inner,
+                          lbytes=2 if w.logit_dtype == "bf16" else 4)
 
     # ---- end to end through the public API: pinned host inputs, copies timed
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(bf).pin_memory()

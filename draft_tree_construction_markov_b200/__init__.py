@@ -21,7 +21,7 @@ __all__ = ["Tree", "tree_build", "tree_verify_attn", "tree_accept", "markov_logi
            "tree_accept_noalloc",
            "shard_range", "shard_cfg", "sharded_workspace_bytes", "sharded_partials_bytes",
            "sharded_build_begin", "sharded_build_gemm", "sharded_build_frontier",
-           "tree_build_sharded"]
+           "tree_build_sharded", "set_build_path", "set_build_wait_test"]
 
 
 def num_sms() -> int:
@@ -267,6 +267,18 @@ def tree_build_sharded(cfg, rank, block_logits, markov_a, markov_b_shard, root_t
         sharded_build_frontier(cfg, wave, gathered, n_budget, lam, out, ws, calib=calib,
                                k_req=k_req, stream=stream)
     return out
+
+
+def set_build_path(path: str) -> None:
+    """How tree_build runs its waves on this host thread: "auto", "waves" or
+    "persistent" (dt_set_build_path)."""
+    _lib.lib.dt_set_build_path(_lib.BUILD_PATHS[path])
+
+
+def set_build_wait_test(stall_cta: int, wait_ns: int) -> None:
+    """Test hook: the next persistent build on this thread stalls one CTA at its
+    first grid barrier and bounds every wait by wait_ns (dt_set_build_wait_test)."""
+    _lib.lib.dt_set_build_wait_test(int(stall_cta), int(wait_ns))
 
 
 def read_status(ws, stream=None) -> int:

@@ -86,8 +86,12 @@ _sig("dt_read_status", _i32, _vp, _vp, ctypes.POINTER(ctypes.c_int32))
 _sig("dt_set_profile_events", None, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int32),
      _i32, ctypes.POINTER(ctypes.c_int32))
 
+_sig("dt_set_build_path", None, _i32)
+_sig("dt_set_build_wait_test", None, _i32, _u64)
+
 KERNEL_KINDS = ["build_init", "markov_gemm", "frontier", "draft_q", "accept_prepass",
-                "accept_walk", "attn", "attn_combine", "other", "tf_lmhead", "tf_mlp"]
+                "accept_walk", "attn", "attn_combine", "other", "tf_lmhead", "tf_mlp", "pbuild"]
+BUILD_PATHS = {"auto": 0, "waves": 1, "persistent": 2}
 
 
 class DtreeError(RuntimeError):

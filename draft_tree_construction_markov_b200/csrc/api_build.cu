@@ -16,6 +16,14 @@ cudaError_t launch_markov_gemm(int mode, bool stoch, const CUtensorMap& tmW,
 cudaError_t launch_frontier(const FrontierArgs& f, cudaStream_t s);
 cudaError_t launch_build_init(const FrontierArgs& f, const int32_t* root_token, Row* rows0,
                               int32_t* count0, cudaStream_t s);
+int pbuild_cols(int batch, int Nmax, int r);
+cudaError_t launch_pbuild(const CUtensorMap& tmW, PBuildArgs a, int ncta, cudaStream_t s);
+
+// How dt_tree_build runs its waves (dt_set_build_path) and the wait-limit
+// test hook (dt_set_build_wait_test); both per host thread.
+static thread_local int g_build_path = DT_BUILD_AUTO;
+static thread_local int g_stall_cta = -1;
+static thread_local uint64_t g_stall_wait_ns = 0;
 
 // ------------------------------------------------------------ profile hook --
 static thread_local void** g_prof_events = nullptr;
@@ -94,6 +102,14 @@ struct BuildLayout {
   int32_t* pli;
   float* pgv;
   int32_t* pgi;
+  // the persistent build alternates two partial buffers by wave parity
+  float2* pstats2;
+  float* plv2;
+  int32_t* pli2;
+  float* pgv2;
+  int32_t* pgi2;
+  unsigned* grid_bar;  // header words 8-10: grid-barrier arrivals, abort flag, exits
+  int32_t* grid_abort;
   int32_t* cond;       // [batch][Bk] per-depth Markov-row tokens of a baseline variant
   int32_t* chain_nb;   // [batch] Shared-Markov chain: node budget min(Bk, n_budget)
   float* chain_lam;    // [batch] Shared-Markov chain: no survival stop
@@ -134,6 +150,13 @@ static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k
   L.pli = c.take<int32_t>(np * k);
   L.pgv = c.take<float>(np * k);
   L.pgi = c.take<int32_t>(np * k);
+  L.pstats2 = c.take<float2>(np);
+  L.plv2 = c.take<float>(np * k);
+  L.pli2 = c.take<int32_t>(np * k);
+  L.pgv2 = c.take<float>(np * k);
+  L.pgi2 = c.take<int32_t>(np * k);
+  L.grid_bar = (unsigned*)(hdr + 8);
+  L.grid_abort = hdr + 9;
   L.cond = c.take<int32_t>((size_t)batch * Bk);
   L.chain_nb = c.take<int32_t>(batch);
   L.chain_lam = c.take<float>(batch);
@@ -246,14 +269,113 @@ static GemmArgs gemm_args(const BuildLayout& L, const void* d_block_logits, dt_d
   // a wave's column count is only known on the device: one CTA per weight
   // range loops over the node tiles that have columns
   g.n_nslots = 1;
+  // every wave of the build streams the same Markov factor: keep it in L2
+  g.l2_keep = 1;
   return g;
 }
 
-// init + Bk waves of GEMM and frontier (+ the draft-q pass at T > 0)
+static dt_status run_wave_launches(FrontierArgs f, GemmArgs g, const BuildLayout& L,
+                                   const int32_t* d_root_token, const CUtensorMap& tmW,
+                                   const CUtensorMap& tmH, int batch, int Bk, cudaStream_t s);
+
+// Arguments of the persistent build, from the wave launches' arguments.
+static PBuildArgs pbuild_args(const FrontierArgs& f, const GemmArgs& g, const BuildLayout& L,
+                              const int32_t* d_root_token) {
+  PBuildArgs a;
+  memset(&a, 0, sizeof(a));
+  a.L = g.L;
+  a.l_bf16 = g.l_bf16;
+  a.A = f.A;
+  a.Bk = f.Bk;
+  a.V = f.V;
+  a.r = f.r;
+  a.k = f.k;
+  a.Nmax = f.Nmax;
+  a.batch = f.batch;
+  a.n_vtiles = L.n_vtiles;
+  a.temp = f.temp;
+  a.seed = g.seed;
+  a.offset = g.offset;
+  a.calib = f.calib;
+  a.root_token = d_root_token;
+  a.n_budget = f.n_budget;
+  a.k_req = f.k_req;
+  a.lambda = f.lambda;
+  a.cond = f.cond;
+  a.pstats[0] = L.pstats;
+  a.plv[0] = L.plv;
+  a.pli[0] = L.pli;
+  a.pgv[0] = L.pgv;
+  a.pgi[0] = L.pgi;
+  a.pstats[1] = L.pstats2;
+  a.plv[1] = L.plv2;
+  a.pli[1] = L.pli2;
+  a.pgv[1] = L.pgv2;
+  a.pgi[1] = L.pgi2;
+  a.grid_bar = L.grid_bar;
+  a.grid_abort = L.grid_abort;
+  a.mat_rows = L.mat_rows;
+  a.mat_count = L.counts + 2;
+  a.out = f.out;
+  a.status = L.status;
+  a.wait_ns = kWaitLimitNs;
+  a.stall_cta = -1;
+  return a;
+}
+
+// init + Bk waves of GEMM and frontier, or one persistent launch for them
+// all (+ the draft-q pass at T > 0)
 static dt_status run_waves(FrontierArgs f, GemmArgs g, const BuildLayout& L,
                            const int32_t* d_root_token, const CUtensorMap& tmW,
                            const CUtensorMap& tmH, const CUtensorMap& tmHm, int batch, int Bk,
                            int Nmax, float* d_draft_q, cudaStream_t s) {
+  const bool fits = pbuild_cols(batch, Nmax, f.r) > 0;
+  if (g_build_path == DT_BUILD_PERSISTENT && !fits) return DT_EUNSUPPORTED;
+  bool waves = g_build_path == DT_BUILD_WAVES || !fits;
+  if (!waves) {
+    PBuildArgs a = pbuild_args(f, g, L, d_root_token);
+    if (g_stall_cta >= 0) {
+      a.stall_cta = g_stall_cta;
+      a.wait_ns = g_stall_wait_ns;
+      g_stall_cta = -1;
+    }
+    cudaError_t e;
+    {
+      ProfileScope ps(DT_K_PBUILD, s);
+      e = launch_pbuild(tmW, a, L.ncta_v, s);
+    }
+    if (e == cudaErrorNotSupported || e == cudaErrorCooperativeLaunchTooLarge) {
+      (void)cudaGetLastError();
+      if (g_build_path == DT_BUILD_PERSISTENT) return DT_EUNSUPPORTED;
+      waves = true;  // nothing was enqueued: run the waves instead
+    } else if (e != cudaSuccess) {
+      return DT_ECUDA;
+    }
+  }
+  if (waves) {
+    const dt_status st = run_wave_launches(f, g, L, d_root_token, tmW, tmH, batch, Bk, s);
+    if (st != DT_OK) return st;
+  }
+  const bool stoch = f.temp > 0.f;
+  if (stoch) {
+    GemmArgs gq = g;
+    gq.rows = L.mat_rows;
+    gq.n_rows = L.counts + 2;
+    gq.reset_count = nullptr;
+    gq.Mcap = L.Mmat;
+    gq.out = d_draft_q;
+    gq.nmax1 = Nmax + 1;
+    ProfileScope ps(DT_K_DRAFT_Q, s);
+    if (launch_markov_gemm(EPI_QROWS, true, tmW, tmW, tmHm, gq, batch, L.nt, s) != cudaSuccess)
+      return DT_ECUDA;
+  }
+  return DT_OK;
+}
+
+// init + Bk waves of GEMM and frontier
+static dt_status run_wave_launches(FrontierArgs f, GemmArgs g, const BuildLayout& L,
+                                   const int32_t* d_root_token, const CUtensorMap& tmW,
+                                   const CUtensorMap& tmH, int batch, int Bk, cudaStream_t s) {
   {
     ProfileScope ps(DT_K_BUILD_INIT, s);
     if (launch_build_init(f, d_root_token, L.rows[0], L.counts + 0, s) != cudaSuccess)
@@ -279,18 +401,6 @@ static dt_status run_waves(FrontierArgs f, GemmArgs g, const BuildLayout& L,
       if (launch_frontier(f, s) != cudaSuccess) return DT_ECUDA;
     }
   }
-  if (stoch) {
-    GemmArgs gq = g;
-    gq.rows = L.mat_rows;
-    gq.n_rows = L.counts + 2;
-    gq.reset_count = nullptr;
-    gq.Mcap = L.Mmat;
-    gq.out = d_draft_q;
-    gq.nmax1 = Nmax + 1;
-    ProfileScope ps(DT_K_DRAFT_Q, s);
-    if (launch_markov_gemm(EPI_QROWS, true, tmW, tmW, tmHm, gq, batch, L.nt, s) != cudaSuccess)
-      return DT_ECUDA;
-  }
   return DT_OK;
 }
 
@@ -309,6 +419,15 @@ using namespace dt;
 extern "C" {
 
 int dt_num_sms(void) { return num_sms(); }
+
+void dt_set_build_path(int path) {
+  g_build_path = (path == DT_BUILD_WAVES || path == DT_BUILD_PERSISTENT) ? path : DT_BUILD_AUTO;
+}
+
+void dt_set_build_wait_test(int stall_cta, uint64_t wait_ns) {
+  g_stall_cta = stall_cta;
+  g_stall_wait_ns = wait_ns;
+}
 
 void dt_set_profile_events(void** events, int32_t* kinds, int capacity, int32_t* count) {
   g_prof_events = events;
@@ -383,7 +502,8 @@ static dt_status build_impl(const void* d_block_logits, dt_dtype ldt, const uint
       !make_tmap_bf16_kmajor(&tmHm, L.Hm, r, L.Mmat_pad, L.nt))
     return DT_ECUDA;
 
-  if (cudaMemsetAsync(L.status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
+  // status, wave counters and the persistent build's grid-barrier words
+  if (cudaMemsetAsync(L.status, 0, 64, s) != cudaSuccess) return DT_ECUDA;
 
   FrontierArgs f = frontier_args(L, d_markov_a, d_calib, d_n_budget, d_k_req, d_lambda, batch,
                                  Bk, V, r, k, Nmax, temp, out);

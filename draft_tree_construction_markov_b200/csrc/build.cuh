@@ -84,6 +84,7 @@ struct GemmArgs {
   int nmax1;             // Nmax + 1
   int32_t* status;
   int stages;
+  int l2_keep;           // weight loads carry an L2 evict-last hint (re-read by later waves)
 };
 
 struct FrontierArgs {
@@ -113,6 +114,41 @@ struct FrontierArgs {
   float temp;
   dt_tree out;
   int32_t* status;
+};
+
+// One persistent launch for every wave of a small build (pbuild.cu).
+struct PBuildArgs {
+  const void* L;          // block logits [batch][Bk][V]
+  int l_bf16;
+  const uint16_t* A;      // Markov rows [V][r] (the MMA's B operand, gathered)
+  int Bk, V, r, k, Nmax, batch;
+  int n_vtiles;           // 128-row tiles of Bm
+  float temp;
+  uint64_t seed;
+  uint32_t offset;
+  const float* calib;     // [Bk][2] or NULL
+  const int32_t* root_token;
+  const int32_t* n_budget;
+  const int32_t* k_req;   // or NULL: k for every request
+  const float* lambda;
+  const int32_t* cond;    // [batch][Bk] Markov-row token per depth of a baseline variant, or NULL
+  // per-CTA partials, two buffers (wave parity); same layout as the wave GEMM's
+  float2* pstats[2];
+  float* plv[2];
+  int32_t* pli[2];
+  float* pgv[2];
+  int32_t* pgi[2];
+  unsigned* grid_bar;     // arrivals so far (zeroed before the launch)
+  int32_t* grid_abort;    // set by a CTA that gave up (zeroed before the launch)
+  Row* mat_rows;          // T > 0: draft rows of the final trees
+  int32_t* mat_count;
+  dt_tree out;
+  int32_t* status;
+  int stages;
+  int span;               // bias cache row length (elements; a multiple of 128)
+  int cap;                // candidate capacity of one request: Nmax + Nmax * k
+  uint64_t wait_ns;       // bound of every device-side wait
+  int stall_cta;          // test hook: this CTA never arrives at the first grid barrier (-1: none)
 };
 
 }  // namespace dt

@@ -279,7 +279,12 @@ dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt,
  *     temporaries; calls that overlap on the GPU race, so serialise them
  *     (e.g. one stream).  Outputs are written to the caller's buffers only.
  *   - Device-side range failures of this variant are not reported through a
- *     readable status word. */
+ *     readable status word.
+ *   - The looked-up address is cached for the life of the process.  After
+ *     cudaDeviceReset (or anything else that destroys and recreates the
+ *     device's primary context) the library's device memory is loaded anew
+ *     and the cached address is stale: do not call this entry point on a
+ *     device after resetting it. */
 dt_status dt_tree_accept_noalloc(const void* d_target_logits, dt_dtype tdt,
                                  const dt_tree* tree, int batch, int Bk, int V,
                                  int Nmax, float temp, uint64_t philox_seed,
@@ -435,8 +440,36 @@ typedef enum {
   DT_K_ATTN_COMBINE = 7,
   DT_K_OTHER = 8,
   DT_K_TF_LMHEAD = 9,     /* TreeFlash LM head + top-M epilogue               */
-  DT_K_TF_MLP = 10        /* TreeFlash SwiGLU / down projection               */
+  DT_K_TF_MLP = 10,       /* TreeFlash SwiGLU / down projection               */
+  DT_K_PBUILD = 11        /* every wave of a small build in one launch        */
 } dt_kernel_kind;
+
+/* How dt_tree_build and dt_tree_build_ex run the waves of the best-first
+ * expansion (TreeSpark article, "core idea"; the exact wave schedule is
+ * described with dt_tree_build).  The result is the same either way; this is
+ * a tuning and diagnostic switch, set per host thread.
+ *   DT_BUILD_AUTO        one persistent launch when batch * Nmax <= 64 and
+ *                        r <= 256 (and the device can hold one such CTA per
+ *                        SM), otherwise one GEMM and one frontier launch per
+ *                        wave (the default);
+ *   DT_BUILD_WAVES       always one launch pair per wave;
+ *   DT_BUILD_PERSISTENT  always the persistent launch: calls that do not fit
+ *                        it return DT_EUNSUPPORTED with nothing enqueued.
+ * The persistent launch is cooperative (all its CTAs are resident at once):
+ * its CTAs meet at a grid barrier after every wave, each wait bounded by two
+ * seconds, after which the call records DT_ETIMEOUT (dt_read_status). */
+typedef enum { DT_BUILD_AUTO = 0, DT_BUILD_WAVES = 1, DT_BUILD_PERSISTENT = 2 } dt_build_path;
+void dt_set_build_path(int path);
+
+/* Test hook for the bounded waits of the persistent build (no counterpart in
+ * the pages).  The next persistent build started from the calling host thread
+ * runs with every device-side wait bounded by wait_ns instead of two seconds,
+ * and its CTA number stall_cta never arrives at the first grid barrier, so
+ * every CTA gives up at that barrier: the call's status becomes DT_ETIMEOUT,
+ * every CTA lets its copies in flight land, frees its tensor memory and
+ * returns, and the tree outputs are left unspecified.  The hook then clears
+ * itself.  stall_cta < 0 clears it without a build. */
+void dt_set_build_wait_test(int stall_cta, uint64_t wait_ns);
 
 /* Profiling hook (measurement only; off by default).  While set, every kernel
  * the library launches from the calling host thread is bracketed by

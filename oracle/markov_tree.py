@@ -15,7 +15,7 @@ are listed with each function):
   * TreeSpark article, "lossless" section: siblings are sampled without
     replacement.
 
-Readings fixed here (each also listed in the design notes):
+Readings fixed here (the pages leave each of these open):
   * temperature: s = z / T for T > 0; at T = 0 tokens are the top-k of z and
     the survival estimate uses T = 1.
   * calibration of child depth d: c_d(l) = min(0, alpha_d * l + beta_d),

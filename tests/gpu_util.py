@@ -24,16 +24,22 @@ def build_inputs(w):
         k_req=dev(w.k_req), calib=None if w.calib is None else dev(np.asarray(w.calib, np.float32)))
 
 
-def run_build(w, temp=None, seed=None, offset=0):
+def run_build(w, temp=None, seed=None, offset=0, path="auto"):
+    """Build the workload's trees; path selects how the waves run ("auto",
+    "waves": one launch pair per wave, "persistent": one launch)."""
     import draft_tree_construction_markov_b200 as dt
     temp = w.temp if temp is None else temp
     x = build_inputs(w)
     tree = dt.Tree.empty(w.batch, w.Nmax, w.V, stochastic=temp > 0)
     ws = dt.workspace(dt.build_workspace_bytes(w.batch, w.Bk, w.V, w.r, w.k, w.Nmax))
-    dt.tree_build(x["block_logits"], x["markov_a"], x["markov_b"], x["root_token"],
-                  x["n_budget"], x["lam"], k=w.k, Nmax=w.Nmax, temp=temp, out=tree, ws=ws,
-                  calib=x["calib"], k_req=x["k_req"],
-                  philox_seed=w.philox_seed if seed is None else seed, philox_offset=offset)
+    dt.set_build_path(path)
+    try:
+        dt.tree_build(x["block_logits"], x["markov_a"], x["markov_b"], x["root_token"],
+                      x["n_budget"], x["lam"], k=w.k, Nmax=w.Nmax, temp=temp, out=tree, ws=ws,
+                      calib=x["calib"], k_req=x["k_req"],
+                      philox_seed=w.philox_seed if seed is None else seed, philox_offset=offset)
+    finally:
+        dt.set_build_path("auto")
     status = dt.read_status(ws)
     assert status == 0, f"device status {status}"
     return tree

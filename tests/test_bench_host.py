@@ -12,9 +12,11 @@ import time
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 FAKE = """#!{py}
-import time
+import datetime, time
 while True:
-    print("0, 1965, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Active", flush=True)
+    ts = datetime.datetime.now().strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+    print("0, 1965, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Active, " + ts,
+          flush=True)
     time.sleep(0.05)
 """
 
@@ -28,11 +30,34 @@ def test_clock_sampler_brackets_a_short_region(tmp_path, monkeypatch):
     import bench
     c = bench.ClockSampler(0)
     c.start()
+    t0 = time.time()
     time.sleep(0.005)   # the timed region
-    r = c.stop()
+    r = c.stop((t0, time.time()))
     assert r is not None and r["samples"] >= 2
     assert r["sm_mhz"] == 1965.0 and r["sm_max_mhz"] == 1965.0
     assert r["reasons"] == ["sw_power_cap"]
+    # shorter than the sampling interval: the samples around it stand in
+    assert r["window"] in ("bracketing", "region")
+
+
+def test_clock_summary_keeps_only_the_region():
+    sys.path.insert(0, ROOT)
+    import bench
+    import datetime
+    base = datetime.datetime(2026, 1, 1, 12, 0, 0)
+    line = lambda s, mhz, cap: (f"0, {mhz}, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, "
+                                f"{cap}, " + (base + datetime.timedelta(seconds=s)).strftime(
+                                    "%Y/%m/%d %H:%M:%S.%f")[:-3])
+    lines = [line(0.0, 1200, "Active"), line(0.5, 1965, "Not Active"), line(0.6, 1965, "Not Active"),
+             line(1.5, 1100, "Active")]
+    t = lambda s: (base + datetime.timedelta(seconds=s)).timestamp()
+    r = bench.summarise_clocks(lines, (t(0.4), t(0.7)))
+    # the throttled samples outside the region do not count
+    assert r["window"] == "region" and r["samples_in_region"] == 2
+    assert r["sm_mhz"] == 1965.0 and r["reasons"] == []
+    r = bench.summarise_clocks(lines, (t(0.7), t(0.8)))   # no sample inside
+    assert r["window"] == "bracketing" and r["samples_in_region"] == 0
+    assert r["sm_mhz"] == (1965.0 + 1100.0) / 2 and r["reasons"] == ["sw_power_cap"]
 
 
 def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
@@ -55,8 +80,11 @@ def test_traffic_is_read_only_for_the_profiled_source(tmp_path, monkeypatch):
     prof = tmp_path / "profiles" / "markov_gemm_qwen3_4b.txt"
     prof.write_text(f"# summary\nsource_sha256_16: {sha}\ndram_bytes_per_launch: 80091904\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.traffic_from_profile(str(src)) == 80091904.0
+    name = "markov_gemm_qwen3_4b.txt"
+    assert bench.traffic_from_profile(str(src), name) == 80091904.0
     src.write_text("// kernel v2\n")          # the kernel changed since the capture
-    assert bench.traffic_from_profile(str(src)) is None
+    assert bench.traffic_from_profile(str(src), name) is None
     prof.unlink()
-    assert bench.traffic_from_profile(str(src)) is None
+    assert bench.traffic_from_profile(str(src), name) is None
+    # each kernel source has its own summary
+    assert bench.PROFILE_OF["pbuild.cu"] == "pbuild_qwen3_4b.txt"

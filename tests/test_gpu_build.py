@@ -90,25 +90,76 @@ CASES = [
 ]
 
 
+# every case fits both ways of running the waves: one persistent launch, or
+# one GEMM + frontier launch pair per wave
+PATHS = ["persistent", "waves"]
+
+
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("name,over,temp", CASES)
 @pytest.mark.parametrize("seed", [0, 1])
-def test_tree_build_parity(name, over, temp, seed):
+def test_tree_build_parity(name, over, temp, seed, path):
     w = make_workload(name, seed=seed, temp=temp, **over)
-    tree = run_build(w, temp=temp, seed=w.philox_seed)
+    tree = run_build(w, temp=temp, seed=w.philox_seed, path=path)
     for b in range(w.batch):
         compare_tree(w, tree, b, temp, w.philox_seed)
 
 
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("temp", [0.0, 1.0])
-def test_batch_budgets_lambda_calibration(temp):
+def test_batch_budgets_lambda_calibration(temp, path):
     w = make_workload("tiny", seed=3, batch=5, V=600, N=12, k=3, temp=temp)
     w.n_budget[:] = np.array([12, 1, 0, 7, 12], np.int32)
     w.k_req[:] = np.array([3, 3, 1, 2, 1], np.int32)
     w.lam[:] = np.array([0.0, 0.0, 0.0, 0.02, 1e-4], np.float32)
     w.calib = np.array([[0.5, -0.1], [1.5, 0.2], [1.0, 0.0], [0.8, -0.3]], np.float32)
-    tree = run_build(w, temp=temp)
+    tree = run_build(w, temp=temp, path=path)
     for b in range(w.batch):
         compare_tree(w, tree, b, temp, w.philox_seed)
+
+
+def test_persistent_build_rejects_what_it_cannot_hold():
+    # batch * Nmax above 64 never runs persistently: forced, the call is refused
+    w = make_workload("tiny", seed=0, batch=3, N=30)
+    x = build_inputs(w)
+    tree = dt.Tree.empty(w.batch, w.Nmax)
+    ws = dt.workspace(dt.build_workspace_bytes(w.batch, w.Bk, w.V, w.r, w.k, w.Nmax))
+    dt.set_build_path("persistent")
+    try:
+        with pytest.raises(dt.DtreeError) as e:
+            dt.tree_build(x["block_logits"], x["markov_a"], x["markov_b"], x["root_token"],
+                          x["n_budget"], x["lam"], k=w.k, Nmax=w.Nmax, temp=0.0, out=tree, ws=ws)
+        assert e.value.code == dt._lib.DT_EUNSUPPORTED
+    finally:
+        dt.set_build_path("auto")
+    tree = run_build(w, temp=0.0)   # "auto" runs it as waves
+    for b in range(w.batch):
+        compare_tree(w, tree, b, 0.0, 0)
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3_4b"])
+def test_persistent_build_wait_runs_out(name):
+    """A CTA that never reaches the first grid barrier: every wait gives up
+    after the test's 1 ms limit, the call reports DT_ETIMEOUT, and the next
+    build on the same stream and workspace is exact again."""
+    w = make_workload(name, seed=2)
+    x = build_inputs(w)
+    tree = dt.Tree.empty(w.batch, w.Nmax)
+    ws = dt.workspace(dt.build_workspace_bytes(w.batch, w.Bk, w.V, w.r, w.k, w.Nmax))
+    args = (x["block_logits"], x["markov_a"], x["markov_b"], x["root_token"], x["n_budget"],
+            x["lam"])
+    dt.set_build_path("persistent")
+    try:
+        dt.set_build_wait_test(0, 1_000_000)
+        dt.tree_build(*args, k=w.k, Nmax=w.Nmax, temp=0.0, out=tree, ws=ws)
+        assert dt.read_status(ws) == dt._lib.DT_ETIMEOUT
+        tree2 = dt.Tree.empty(w.batch, w.Nmax)
+        dt.tree_build(*args, k=w.k, Nmax=w.Nmax, temp=0.0, out=tree2, ws=ws)
+        assert dt.read_status(ws) == 0
+    finally:
+        dt.set_build_wait_test(-1, 0)
+        dt.set_build_path("auto")
+    compare_tree(w, tree2, 0, 0.0, 0)
 
 
 def test_k1_is_greedy_chain_on_gpu():

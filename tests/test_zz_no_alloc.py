@@ -21,12 +21,14 @@ if torch.cuda.is_available():
     from draft_tree_construction_markov_b200 import _lib
     from tests.gpu_util import BF16, dev, run_build, target_for_tree, tree_to_host
 
+    # the C entry point with the signature the binding declares for it (checked
+    # here, not reassigned, so the binding's own declaration is what runs)
     _fn = _lib.lib.dt_tree_accept_noalloc
-    _fn.restype = ctypes.c_int
-    _fn.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(_lib.DtTree), ctypes.c_int,
-                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_uint64,
-                    ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                    ctypes.c_void_p]
+    assert _fn.restype is ctypes.c_int
+    assert list(_fn.argtypes) == [
+        ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(_lib.DtTree), ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64,
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
 
 
 def _outputs(w):
