@@ -17,7 +17,7 @@ cudaError_t launch_frontier(const FrontierArgs& f, cudaStream_t s);
 cudaError_t launch_build_init(const FrontierArgs& f, const int32_t* root_token, Row* rows0,
                               int32_t* count0, cudaStream_t s);
 int pbuild_cols(int batch, int Nmax, int r);
-cudaError_t launch_pbuild(const CUtensorMap& tmW, PBuildArgs a, int ncta, cudaStream_t s);
+cudaError_t launch_pbuild(const uint16_t* d_markov_b, PBuildArgs a, int ncta, cudaStream_t s);
 
 // How dt_tree_build runs its waves (dt_set_build_path) and the wait-limit
 // test hook (dt_set_build_wait_test); both per host thread.
@@ -108,6 +108,9 @@ struct BuildLayout {
   int32_t* pli2;
   float* pgv2;
   int32_t* pgi2;
+  float* mrg_lse;      // merged rows of a persistent-build wave
+  float* mrg_val;
+  int32_t* mrg_tok;
   unsigned* grid_bar;  // header words 8-10: grid-barrier arrivals, abort flag, exits
   int32_t* grid_abort;
   int32_t* cond;       // [batch][Bk] per-depth Markov-row tokens of a baseline variant
@@ -155,6 +158,9 @@ static BuildLayout build_layout(void* ws, int batch, int Bk, int V, int r, int k
   L.pli2 = c.take<int32_t>(np * k);
   L.pgv2 = c.take<float>(np * k);
   L.pgi2 = c.take<int32_t>(np * k);
+  L.mrg_lse = c.take<float>(L.Mcap);
+  L.mrg_val = c.take<float>((size_t)L.Mcap * k);
+  L.mrg_tok = c.take<int32_t>((size_t)L.Mcap * k);
   L.grid_bar = (unsigned*)(hdr + 8);
   L.grid_abort = hdr + 9;
   L.cond = c.take<int32_t>((size_t)batch * Bk);
@@ -312,6 +318,9 @@ static PBuildArgs pbuild_args(const FrontierArgs& f, const GemmArgs& g, const Bu
   a.pli[1] = L.pli2;
   a.pgv[1] = L.pgv2;
   a.pgi[1] = L.pgi2;
+  a.mrg_lse = L.mrg_lse;
+  a.mrg_val = L.mrg_val;
+  a.mrg_tok = L.mrg_tok;
   a.grid_bar = L.grid_bar;
   a.grid_abort = L.grid_abort;
   a.mat_rows = L.mat_rows;
@@ -326,7 +335,8 @@ static PBuildArgs pbuild_args(const FrontierArgs& f, const GemmArgs& g, const Bu
 // init + Bk waves of GEMM and frontier, or one persistent launch for them
 // all (+ the draft-q pass at T > 0)
 static dt_status run_waves(FrontierArgs f, GemmArgs g, const BuildLayout& L,
-                           const int32_t* d_root_token, const CUtensorMap& tmW,
+                           const int32_t* d_root_token, const uint16_t* d_markov_b,
+                           const CUtensorMap& tmW,
                            const CUtensorMap& tmH, const CUtensorMap& tmHm, int batch, int Bk,
                            int Nmax, float* d_draft_q, cudaStream_t s) {
   const bool fits = pbuild_cols(batch, Nmax, f.r) > 0;
@@ -342,7 +352,7 @@ static dt_status run_waves(FrontierArgs f, GemmArgs g, const BuildLayout& L,
     cudaError_t e;
     {
       ProfileScope ps(DT_K_PBUILD, s);
-      e = launch_pbuild(tmW, a, L.ncta_v, s);
+      e = launch_pbuild(d_markov_b, a, L.ncta_v, s);
     }
     if (e == cudaErrorNotSupported || e == cudaErrorCooperativeLaunchTooLarge) {
       (void)cudaGetLastError();
@@ -533,7 +543,7 @@ static dt_status build_impl(const void* d_block_logits, dt_dtype ldt, const uint
     fc.lambda = L.chain_lam;
     fc.temp = 0.f;
     gc.temp = 0.f;
-    const dt_status st = run_waves(fc, gc, L, d_root_token, tmW, tmH, tmHm, batch, Bk, Nmax,
+    const dt_status st = run_waves(fc, gc, L, d_root_token, d_markov_b, tmW, tmH, tmHm, batch, Bk, Nmax,
                                    nullptr, s);
     if (st != DT_OK) return st;
     {
@@ -544,7 +554,8 @@ static dt_status build_impl(const void* d_block_logits, dt_dtype ldt, const uint
     }
     f.cond = L.cond;
   }
-  return run_waves(f, g, L, d_root_token, tmW, tmH, tmHm, batch, Bk, Nmax, out->d_draft_q, s);
+  return run_waves(f, g, L, d_root_token, d_markov_b, tmW, tmH, tmHm, batch, Bk, Nmax,
+                   out->d_draft_q, s);
 }
 
 }  // namespace dt

@@ -138,6 +138,9 @@ struct PBuildArgs {
   int32_t* pli[2];
   float* pgv[2];
   int32_t* pgi[2];
+  float* mrg_lse;         // merged rows of a wave: log-sum-exp [rows]
+  float* mrg_val;         //   the k best values of s [rows][k]
+  int32_t* mrg_tok;       //   their tokens (T = 0) or the sampled tokens (T > 0) [rows][k]
   unsigned* grid_bar;     // arrivals so far (zeroed before the launch)
   int32_t* grid_abort;    // set by a CTA that gave up (zeroed before the launch)
   Row* mat_rows;          // T > 0: draft rows of the final trees

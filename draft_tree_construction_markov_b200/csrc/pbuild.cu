@@ -38,19 +38,35 @@
 
 namespace dt {
 
+// Roles of the 10 warps.  The nodes of a wave are the rows of the MMA's A
+// operand (M = 128) and the streamed Bm tiles the B operand, 256 vocabulary
+// rows per MMA.  tcgen05.ld lets warp w read TMEM lane quadrant w % 4 only,
+// and the four quadrants belong to the SM's four sub-partitions.  So that
+// the epilogue runs on all four, the NT node rows are replicated R = 128 / NT
+// times down the A operand (the MMA computes every replica at no extra
+// cost): quadrant q holds node group q % (NT / 32) of replica q / (NT / 32).
+// Epilogue warps 0-7 (two per quadrant) split a tile's 256 columns: the
+// 2R warps that see the same node group take one part of 256 / (2R) = NT
+// columns each.
 template <int NG>
 struct PShape {
-  static constexpr int NT = 32 * NG;          // MMA N: node columns (one tile per wave)
-  static constexpr int kEpiWarps = 4 * NG;    // one warp per (TMEM quadrant, 32 columns)
-  static constexpr int kThreads = 32 * (2 + kEpiWarps);
+  static constexpr int NT = 32 * NG;          // node rows per replica
+  static constexpr int R = 4 / NG;            // replicas down the 128 A rows
+  static constexpr int kThreads = 320;
+  static constexpr int kEpiWarps = 8;         // warps 0-7
+  static constexpr int kWarpMma = 8;
+  static constexpr int kWarpProd = 9;
+  static constexpr int kParts = 2 * R;        // column parts of a tile per node group
+  static constexpr int kPartCols = 256 / kParts;  // = NT
   static constexpr int kCompute = kThreads - 32;  // every warp but the producer
   static constexpr int kCWarps = kCompute / 32;
-  static constexpr int kAccBufs = 4;
-  static constexpr uint32_t kTmemCols = kAccBufs * NT;  // 128 or 256
-  static constexpr int kABytes = kTileV * 128;          // 128 weight rows x 64 bf16
-  static_assert(NG == 1 || NG == 2, "32 or 64 node columns");
+  static constexpr int kMergeWarps = 4;       // warps of a CTA that merge node rows
+  static constexpr int kTileN = 256;          // vocabulary rows per MMA tile
+  static constexpr int kStageBytes = kTileN * 128;  // 256 rows x 64 bf16 of Bm
+  static constexpr int kAccBufs = 2;          // TMEM accumulators of 128 x 256 fp32
+  static constexpr uint32_t kTmemCols = kAccBufs * kTileN;  // the whole TMEM
+  static_assert(NG == 1 || NG == 2, "32 or 64 node rows");
 };
-
 
 // Column of this wave's tile as the epilogue sees it.
 struct PMeta {
@@ -63,47 +79,31 @@ struct PMeta {
 
 // Shared-memory layout, computed the same way on the host (size) and the
 // device (offsets).  Offsets are from a 1024-byte aligned base.
+//
+// The A operand: chunk kc (K columns 64 kc .. 64 kc + 63) of A row i at
+// a + (kc * 128 + i) * 128, 128-byte swizzled; A row i holds node i % NT.
 struct PLayout {
-  size_t stage, bres, bars, flags, rows0, rows1, meta, tbuf, bias, req, lists, cands, sorted,
-      keys, rlse, rlq, rtok, spos, spar, msv, msi, misc, total;
+  size_t a, bias, lists, cands, sorted, keys, rlse, rlq, rtok, spos, spar, msv, msi, misc, req,
+      rows0, rows1, meta, exch, bars, flags, stage, total;
 };
 
 __host__ __device__ inline size_t p_align(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Elements per row of the bias cache: the CTA's vocabulary range (span) plus
+// 16 bytes, so that the rows of different depths start in different banks.
+__host__ __device__ inline int p_bias_stride(int span, int esz) { return span + 16 / esz; }
 
 template <int NG>
 __host__ __device__ inline PLayout p_layout(int stages, int r, int k, int Nmax, int batch, int Bk,
                                             int span, int esz, int kmax, bool stoch) {
   using S = PShape<NG>;
+  const int KC = (r + 63) / 64;
   PLayout l;
   size_t o = 0;
-  l.stage = o;
-  o += (size_t)stages * S::kABytes;
-  l.bres = o;
-  o += (size_t)((r + 63) / 64) * S::NT * 128;
-  l.bars = o;
-  o += (size_t)(2 * stages + 2 * S::kAccBufs + 1) * 8;  // + the MMA drain barrier
-  l.flags = o;
-  o += 16;
-  o = p_align(o, 32);
-  l.rows0 = o;
-  o += (size_t)S::NT * sizeof(Row);
-  l.rows1 = o;
-  o += (size_t)S::NT * sizeof(Row);
-  l.meta = o;
-  o += (size_t)S::NT * sizeof(PMeta);
-  o = p_align(o, 16);
-  l.tbuf = o;
-  {
-    const size_t tb = (size_t)S::kEpiWarps * 32 * kTLD * 4;
-    const size_t lists = (size_t)4 * S::NT * kmax * 8 * (stoch ? 2 : 1) + (size_t)4 * S::NT * 8;
-    o += tb > lists ? tb : lists;
-  }
-  o = p_align(o, 16);
+  l.a = o;
+  o += (size_t)KC * 128 * 128;
   l.bias = o;
-  o += (size_t)batch * Bk * span * esz;
-  o = p_align(o, 16);
-  l.req = o;
-  o += (size_t)batch * sizeof(ReqState);
+  o += (size_t)batch * Bk * p_bias_stride(span, esz) * esz;
   o = p_align(o, 16);
   l.lists = o;
   o += (size_t)batch * Nmax * sizeof(Cand);
@@ -113,6 +113,14 @@ __host__ __device__ inline PLayout p_layout(int stages, int r, int k, int Nmax, 
   o += (size_t)Nmax * sizeof(Cand);
   l.keys = o;
   o += (size_t)(Nmax + Nmax * k) * 8;
+  // the epilogue's exchange of every column part's per-node partial shares
+  // these bytes with the selection scratch: within a wave the epilogue is
+  // done with it before the selection starts, and vice versa
+  l.exch = l.cands;
+  {
+    const size_t ex = (size_t)S::kParts * S::NT * (8 + (size_t)kmax * 8 * (stoch ? 2 : 1));
+    if (o < l.cands + ex) o = l.cands + ex;
+  }
   l.rlse = o;
   o += (size_t)S::NT * 4;
   l.rlq = o;
@@ -124,11 +132,29 @@ __host__ __device__ inline PLayout p_layout(int stages, int r, int k, int Nmax, 
   l.spar = o;
   o += (size_t)Nmax * 4;
   l.msv = o;
-  o += (size_t)S::kCWarps * 32 * 4;
+  o += (size_t)S::kMergeWarps * 32 * 4;
   l.msi = o;
-  o += (size_t)S::kCWarps * 32 * 4;
+  o += (size_t)S::kMergeWarps * 32 * 4;
   l.misc = o;
   o += 16 * 4;
+  o = p_align(o, 16);
+  l.req = o;
+  o += (size_t)batch * sizeof(ReqState);
+  o = p_align(o, 32);
+  l.rows0 = o;
+  o += (size_t)S::NT * sizeof(Row);
+  l.rows1 = o;
+  o += (size_t)S::NT * sizeof(Row);
+  l.meta = o;
+  o += (size_t)S::NT * sizeof(PMeta);
+  o = p_align(o, 8);
+  l.bars = o;
+  o += (size_t)(2 * stages + 2 * S::kAccBufs + 2) * 8;  // + MMA drain, prefetch gate
+  l.flags = o;
+  o += 16;
+  o = p_align(o, 1024);
+  l.stage = o;
+  o += (size_t)stages * S::kStageBytes;
   l.total = o;
   return l;
 }
@@ -140,7 +166,7 @@ __device__ __forceinline__ bool p_wait(uint64_t* bar, uint32_t parity, const PBu
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > a.wait_ns) {
       *abort_flag = 1;
@@ -430,7 +456,8 @@ namespace dt {
 
 template <int NG, bool STOCH, int KMAX>
 __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
-    pbuild_kernel(const __grid_constant__ CUtensorMap tmW, const PBuildArgs a) {
+    pbuild_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmW128,
+                  const PBuildArgs a) {
   using S = PShape<NG>;
   constexpr int NT = S::NT, NCT = S::kCompute;
   extern __shared__ uint8_t smem_raw[];
@@ -439,20 +466,24 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
   const int esz = a.l_bf16 ? 2 : 4;
   const PLayout lay =
       p_layout<NG>(a.stages, a.r, a.k, a.Nmax, a.batch, a.Bk, a.span, esz, KMAX, STOCH);
+  const int bstride = p_bias_stride(a.span, esz);
+  uint8_t* aop = smem + lay.a;  // node rows A[token]: [KC][NT][128 B], 128-byte swizzle
   uint8_t* stage_mem = smem + lay.stage;
-  uint8_t* bres = smem + lay.bres;  // gathered rows A[token]: [KC][NT][128 B], 128-byte swizzle
   uint64_t* full = (uint64_t*)(smem + lay.bars);
   uint64_t* empty = full + a.stages;
   uint64_t* tfull = empty + a.stages;
   uint64_t* tempty = tfull + S::kAccBufs;
+  uint64_t* drain = tempty + S::kAccBufs;
   uint32_t* tmem_slot = (uint32_t*)(smem + lay.flags);
   volatile int* abort_flag = (volatile int*)(smem + lay.flags + 4);
   volatile int* done_flag = (volatile int*)(smem + lay.flags + 8);
+  // pass w >= 1 of the producer (the weights of wave w) starts once phase
+  // w - 1 of this barrier is complete: the compute warps complete one phase
+  // per wave, after reading that wave's merged rows
+  uint64_t* gate = drain + 1;
   Row* rows_buf[2] = {(Row*)(smem + lay.rows0), (Row*)(smem + lay.rows1)};
   PMeta* meta = (PMeta*)(smem + lay.meta);
-  float* tbuf = (float*)(smem + lay.tbuf);
-  uint8_t* bias_cache = smem + lay.bias;  // [batch * Bk][span], the element type of L
-  ReqState* reqs = (ReqState*)(smem + lay.req);
+  uint8_t* bias_cache = smem + lay.bias;  // [batch * Bk][bstride], the element type of L
   Cand* lists = (Cand*)(smem + lay.lists);
   Cand* cands = (Cand*)(smem + lay.cands);
   Cand* sorted = (Cand*)(smem + lay.sorted);
@@ -464,20 +495,26 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
   int* s_par = (int*)(smem + lay.spar);
   float* msv = (float*)(smem + lay.msv);
   int32_t* msi = (int32_t*)(smem + lay.msi);
+  float* exch = (float*)(smem + lay.exch);
   // misc: [0] kept count, [1] next-wave rows, [2] draft rows, [3] waiting rows of
   // a request, [4] its base, [5] rows of this wave, [6] abort snapshot
   int* misc = (int*)(smem + lay.misc);
+  ReqState* reqs = (ReqState*)(smem + lay.req);
 
   const int cx = blockIdx.x, ncta = gridDim.x;
   const bool writer = cx == 0;
+  // this CTA's range: 128-row tiles [t0, t0 + n128), as MMA tiles of 256 rows
+  // (and one of 128 rows when n128 is odd)
   const int base_t = a.n_vtiles / ncta, extra = a.n_vtiles % ncta;
   const int t0 = cx * base_t + min(cx, extra);
-  const int ntile = base_t + (cx < extra ? 1 : 0);
+  const int n128 = base_t + (cx < extra ? 1 : 0);
+  const int n_mt = (n128 + 1) >> 1;
+  const bool odd = (n128 & 1) != 0;
   const int KC = (a.r + 63) >> 6;
   const int ks_last = (((a.r - 1) & 63) >> 4) + 1;
-  const int per_wave = ntile * KC;  // stages of one pass over this CTA's range
+  const int per_wave = n_mt * KC;  // stages of one pass over this CTA's range
   const int x0 = t0 * kTileV;
-  const int x1 = min((t0 + ntile) * kTileV, a.V);
+  const int x1 = min((t0 + n128) * kTileV, a.V);
   const int k = a.k;
 
   if (threadIdx.x == 0) {
@@ -489,13 +526,17 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], S::kEpiWarps);
     }
-    mbar_init(tempty + S::kAccBufs, 1);  // MMA drain
+    mbar_init(drain, 1);
+    mbar_init(gate, 1);
     *abort_flag = 0;
     *done_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tmap(&tmW);
-  if (warp == 1) {
+  if (warp == S::kWarpProd && lane == 0) {
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmW128);
+  }
+  if (warp == S::kWarpMma) {
     tmem_alloc(tmem_slot, S::kTmemCols);
     tc_fence_before();
   }
@@ -503,7 +544,7 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == S::kWarpProd) {
     // ---------------------------------------------------------------- producer
     // Streams this CTA's range of Bm over and over, one pass per wave, as
     // far ahead as the ring allows; stops when the build is over.
@@ -516,7 +557,7 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
         bool got = mbar_try_wait(&empty[stage], ph ^ 1);
         if (!got) {
           const uint64_t tw = globaltimer_ns();
-          while (!(got = mbar_try_wait(&empty[stage], ph ^ 1))) {
+          while (!(got = mbar_try_wait_sleep(&empty[stage], ph ^ 1))) {
             if (*done_flag || *abort_flag) break;
             if (globaltimer_ns() - tw > a.wait_ns) {
               *abort_flag = 1;
@@ -528,10 +569,29 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
         }
         if (!got || *done_flag || *abort_flag) break;
         const int i = (int)(g % (uint32_t)per_wave);
-        const int t = t0 + i / KC, kc = i % KC;
-        uint8_t* sa = stage_mem + (size_t)stage * S::kABytes;
-        mbar_arrive_expect_tx(&full[stage], S::kABytes);
-        tma_load_2d_hint(sa, &tmW, &full[stage], kc * 64, t * kTileV, pol);
+        if (i == 0 && g > 0) {
+          // a pass starts only when the compute warps open it: the merge's
+          // global loads of the previous wave must not queue behind it
+          const uint32_t pass = g / (uint32_t)per_wave;
+          const uint64_t tw = globaltimer_ns();
+          bool open = false;
+          while (!(open = mbar_try_wait_sleep(gate, (pass - 1) & 1u))) {
+            if (*done_flag || *abort_flag) break;
+            if (globaltimer_ns() - tw > a.wait_ns) {
+              *abort_flag = 1;
+              set_status(a.status, DT_ETIMEOUT);
+              atomicExch(a.grid_abort, 1);
+              break;
+            }
+          }
+          if (!open || *done_flag || *abort_flag) break;
+        }
+        const int j = i / KC, kc = i % KC;
+        const bool half = odd && j == n_mt - 1;  // the 128-row tile
+        const int y = (t0 + 2 * j) * kTileV;
+        uint8_t* sa = stage_mem + (size_t)stage * S::kStageBytes;
+        mbar_arrive_expect_tx(&full[stage], half ? S::kStageBytes / 2 : S::kStageBytes);
+        tma_load_2d_hint(sa, half ? &tmW128 : &tmW, &full[stage], kc * 64, y, pol);
         issued |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (ph << stage);
       }
@@ -545,7 +605,8 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
       }
     }
   } else {
-    const int ct = threadIdx.x - 32;
+    // every warp but the producer; ct numbers their threads
+    const int ct = threadIdx.x < 32 * S::kWarpProd ? threadIdx.x : threadIdx.x - 32;
     // ---------------------------------------------------------------- set-up
     // block-logit rows of every (request, depth) over [x0, x1), once
     {
@@ -556,7 +617,7 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
         const int np = nx * esz / 16;  // whole: x0 and V are multiples of 16 bytes here
         for (int idx = ct; idx < nrow * np; idx += NCT) {
           const int u = idx / np, i = idx % np;
-          cp_async16_g2s(bias_cache + ((size_t)u * a.span * esz + (size_t)i * 16),
+          cp_async16_g2s(bias_cache + ((size_t)u * bstride * esz + (size_t)i * 16),
                          (const uint8_t*)a.L + ((size_t)u * a.V + x0) * esz + (size_t)i * 16);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -564,10 +625,10 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
         for (int idx = ct; idx < nrow * nx; idx += NCT) {
           const int u = idx / nx, i = idx % nx;
           if (esz == 2)
-            ((uint16_t*)bias_cache)[(size_t)u * a.span + i] =
+            ((uint16_t*)bias_cache)[(size_t)u * bstride + i] =
                 ((const uint16_t*)a.L)[(size_t)u * a.V + x0 + i];
           else
-            ((float*)bias_cache)[(size_t)u * a.span + i] =
+            ((float*)bias_cache)[(size_t)u * bstride + i] =
                 ((const float*)a.L)[(size_t)u * a.V + x0 + i];
         }
       }
@@ -635,15 +696,16 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
     }
 
     // pipeline positions carried across waves by the threads that own them
-    int m_stage = 0, m_ab = 0, e_ab = 0;
-    uint32_t m_phase = 0, m_aphase = 0, e_aphase = 0;
+    int m_stage = 0;
+    uint32_t m_phase = 0, m_tile = 0, e_tile = 0;  // tile n uses accumulator n % kAccBufs
+    const int cw = warp < S::kWarpProd ? warp : warp - 1;  // compute-warp index
     int cur = 0;
     for (int wave = 0;; ++wave) {
       named_bar(1, NCT);
       const int n_rows = misc[5];
       if (n_rows == 0 || misc[6]) break;  // uniform (shared memory after a barrier)
       Row* rows = rows_buf[cur];
-      // ---- columns of this wave, and their rows A[token] as the MMA's B operand
+      // ---- this wave's node rows, and their Markov rows A[token] as the A operand
       for (int c = ct; c < NT; c += NCT) {
         PMeta m;
         m.valid = 0;
@@ -668,6 +730,7 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
       }
       named_bar(1, NCT);
       {
+        // rows 0 .. NT-1 of every chunk from global memory
         const int npieces = KC * NT * 8;
         for (int idx = ct; idx < npieces; idx += NCT) {
           const int ch = idx & 7, c = (idx >> 3) % NT, kc = (idx >> 3) / NT;
@@ -675,35 +738,55 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
           const int tok = c < n_rows ? rows[c].token : -1;
           const bool ok = meta[c].valid && tok >= 0 && col_k < a.r;
           const uint16_t* src = ok ? a.A + (size_t)tok * a.r + col_k : a.A;
-          uint8_t* dst = bres + ((size_t)kc * NT + c) * 128 + ((ch ^ (c & 7)) << 4);
+          uint8_t* dst = aop + ((size_t)kc * 128 + c) * 128 + ((ch ^ (c & 7)) << 4);
           asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),
                        "l"(src), "r"(ok ? 16 : 0)
                        : "memory");
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         asm volatile("cp.async.wait_all;" ::: "memory");
+      }
+      named_bar(1, NCT);
+      {
+        // A row i (of 128) is node i % NT: the replicas are byte copies of
+        // rows 0 .. NT-1 (NT is a multiple of the 8-row swizzle period)
+        constexpr int per = NT * 128 / 16;  // 16-byte pieces of one replica of a chunk
+        const int n = KC * (S::R - 1) * per;
+        for (int idx = ct; idx < n; idx += NCT) {
+          const int kc = idx / ((S::R - 1) * per);
+          const int rr = 1 + (idx / per) % (S::R - 1);
+          const int pc = idx % per;
+          const uint4* src = (const uint4*)(aop + (size_t)kc * 128 * 128) + pc;
+          uint4* dst = (uint4*)(aop + (size_t)kc * 128 * 128 + (size_t)rr * NT * 128) + pc;
+          *dst = *src;
+        }
         // the tensor cores read these bytes through the async proxy
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       named_bar(1, NCT);
-      if (warp == 1) {
+      if (warp == S::kWarpMma) {
         // ---------------------------------------------------------- MMA issuer
+        // D[i][x] (+)= A[i][k] . Bm[x][k] over the K chunks of a tile:
+        // M = 128 rows (R replicas of the NT node rows), N = 256 vocabulary rows.
         if (lane == 0) {
-          constexpr uint32_t idesc = idesc_bf16_f32(kTileV, NT);
+          constexpr uint32_t idesc_full = idesc_bf16_f32(kTileV, S::kTileN);
+          constexpr uint32_t idesc_half = idesc_bf16_f32(kTileV, S::kTileN / 2);
           bool ok = true;
-          for (int t = 0; t < ntile && ok; ++t) {
-            if (!p_wait(&tempty[m_ab], m_aphase ^ 1, a, abort_flag)) break;
+          for (int j = 0; j < n_mt && ok; ++j) {
+            const int ab = (int)(m_tile % S::kAccBufs);
+            if (!p_wait(&tempty[ab], ((m_tile / S::kAccBufs) & 1u) ^ 1u, a, abort_flag)) break;
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + (uint32_t)(m_ab * NT);
+            const uint32_t idesc = (odd && j == n_mt - 1) ? idesc_half : idesc_full;
+            const uint32_t d_tmem = tmem_base + (uint32_t)(ab * S::kTileN);
             for (int kc = 0; kc < KC; ++kc) {
               if (!p_wait(&full[m_stage], m_phase, a, abort_flag)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-              const uint64_t da =
-                  smem_desc_k_sw128(smem_u32(stage_mem + (size_t)m_stage * S::kABytes));
-              const uint64_t db = smem_desc_k_sw128(smem_u32(bres + (size_t)kc * NT * 128));
+              const uint64_t da = smem_desc_k_sw128(smem_u32(aop + (size_t)kc * 128 * 128));
+              const uint64_t db =
+                  smem_desc_k_sw128(smem_u32(stage_mem + (size_t)m_stage * S::kStageBytes));
               const int ks = (kc == KC - 1) ? ks_last : 4;
               for (int s = 0; s < ks; ++s)
                 tc_mma_bf16(d_tmem, da + 2 * s, db + 2 * s, idesc, (kc | s) != 0 ? 1u : 0u);
@@ -714,27 +797,24 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
               }
             }
             if (!ok) break;
-            tc_commit(&tfull[m_ab]);
-            if (++m_ab == S::kAccBufs) {
-              m_ab = 0;
-              m_aphase ^= 1;
-            }
+            tc_commit(&tfull[ab]);
+            ++m_tile;
           }
         }
         __syncwarp();
-      } else {
-        // ------------------------------------------ epilogue (node columns)
-        // Each 32 x 32 accumulator block (32 vocabulary rows of quadrant q,
-        // 32 node columns) is transposed through the warp's buffer so that
-        // lane c owns column c; per column: bias from the cache, 1/T, an
-        // online max / sum-exp, the top-k of s (ties to the lower token) and,
-        // at T > 0, the Gumbel-top-k of s + G.
-        const int e = warp - 2;
-        const int q = warp & 3;  // TMEM lane quadrant of this warp
-        const int eg = e >> 2;   // its 32-column group
+      } else if (warp < S::kEpiWarps) {
+        // ------------------------------------------------ epilogue (node rows)
+        // Lane = node 32 g + lane of node group g, in quadrant q (replica
+        // q / NG); this warp reduces column part p of every tile (NT columns,
+        // in blocks of 32 read straight from TMEM).  Per node: bias from the
+        // cache, 1/T, an online max / sum-exp, the top-k of s (ties to the
+        // lower token) and, at T > 0, the Gumbel-top-k of s + G.
+        const int q = warp & 3;
+        const int c = 32 * (q % NG) + lane;
+        const int part = (q / NG) * 2 + (warp >> 2);
         const float temp = a.temp;
-        float* tb = tbuf + (size_t)e * 32 * kTLD;
-        const PMeta mc = meta[eg * 32 + lane];
+        const PMeta mc = meta[c];
+        const bool any = __any_sync(0xffffffffu, mc.valid) != 0;
         float m = -INFINITY, ssum = 0.f, thr = -INFINITY, gthr = -INFINITY;
         float L1[KMAX], L2[KMAX];
         int32_t I1[KMAX], I2[KMAX];
@@ -743,166 +823,187 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
           L1[i] = L2[i] = -INFINITY;
           I1[i] = I2[i] = 0x7fffffff;
         }
-        for (int t = 0; t < ntile; ++t) {
+        for (int j = 0; j < n_mt; ++j) {
           // one lane waits; the warp follows it as one (tcgen05.ld is warp-wide)
           __syncwarp();
+          const int ab = (int)(e_tile % S::kAccBufs);
           int ok = 1;
-          if (lane == 0) ok = p_wait(&tfull[e_ab], e_aphase, a, abort_flag) ? 1 : 0;
+          if (lane == 0) ok = p_wait(&tfull[ab], (e_tile / S::kAccBufs) & 1u, a, abort_flag) ? 1 : 0;
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
           tc_fence_after();
-          const int xq = (t0 + t) * kTileV + 32 * q;  // first vocabulary row of the quadrant
-          const int nv = min(32, a.V - xq);
-          float acc[32];
-          tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(e_ab * NT + eg * 32), acc);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[e_ab]);
-          if (++e_ab == S::kAccBufs) {
-            e_ab = 0;
-            e_aphase ^= 1;
-          }
+          // the 128-row tile at the end of an odd range has columns 0-127 only
+          const bool has_part = !(odd && j == n_mt - 1) || part * S::kPartCols < kTileV;
+          if (any && has_part) {
+#pragma unroll 1
+            for (int c4 = 0; c4 < S::kPartCols / 32; ++c4) {
+              __syncwarp();
+              const int col = part * S::kPartCols + 32 * c4;  // within the tile
+              const int xq = (t0 + 2 * j) * kTileV + col;    // first token of the block
+              const int nv = min(32, a.V - xq);
+              float acc[32];
+              tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * S::kTileN + col),
+                        acc);
+              if (!mc.valid || nv <= 0) continue;
+              float bias[32];
+              const size_t ci = (size_t)mc.bslot * bstride + (size_t)(xq - x0);
+              if (nv == 32) {
+                uint4 cr[8];
+                const uint4* src = (const uint4*)(bias_cache + ci * esz);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) tb[lane * kTLD + i] = acc[i];
-          __syncwarp();
+                for (int cc = 0; cc < 8; ++cc)
+                  if (cc < 4 || !a.l_bf16) cr[cc] = src[cc];
+                decode_bias(cr, a.l_bf16, bias);
+              } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[i] = tb[i * kTLD + lane];
-          __syncwarp();
-          if (!mc.valid || nv <= 0) continue;
-          float bias[32];
-          const size_t ci = (size_t)mc.bslot * a.span + (size_t)(xq - x0);
-          if (nv == 32) {
-            uint4 cr[8];
-            const uint4* src = (const uint4*)(bias_cache + ci * esz);
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              if (c < 4 || !a.l_bf16) cr[c] = src[c];
-            decode_bias(cr, a.l_bf16, bias);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              bias[i] = i < nv ? (a.l_bf16 ? bf16_to_f32(((const uint16_t*)bias_cache)[ci + i])
-                                           : ((const float*)bias_cache)[ci + i])
-                               : 0.f;
-          }
-          float s[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float z = acc[i] + bias[i];
-            s[i] = i < nv ? (STOCH ? __fdiv_rn(z, temp) : z) : -INFINITY;
-          }
-          float mx[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) mx[i] = fmaxf(s[i], s[i + 16]);
-#pragma unroll
-          for (int w = 8; w; w >>= 1)
-#pragma unroll
-            for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
-          const float mt = mx[0];
-          float ex[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ex[i] = ex2_approx((s[i] - mt) * kLog2e);
-#pragma unroll
-          for (int w = 16; w; w >>= 1)
-#pragma unroll
-            for (int i = 0; i < w; ++i) ex[i] += ex[i + w];
-          const float st = ex[0];
-          if (mt > m) {
-            ssum = ssum * ex2_approx((m - mt) * kLog2e) + st;
-            m = mt;
-          } else {
-            ssum += st * ex2_approx((mt - m) * kLog2e);
-          }
-          if (mt > thr) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (s[i] > thr) {
-                topk_insert<KMAX>(L1, I1, s[i], xq + i);
-                thr = kth<KMAX>(L1, k);
+                for (int i = 0; i < 32; ++i)
+                  bias[i] = i < nv ? (a.l_bf16 ? bf16_to_f32(((const uint16_t*)bias_cache)[ci + i])
+                                               : ((const float*)bias_cache)[ci + i])
+                                   : 0.f;
               }
-            }
-          }
-          if constexpr (STOCH) {
-            // Gumbel keys; four consecutive tokens share one Philox counter
-            if (mt + kGumbelMax > gthr) {
+              float sv[32];
 #pragma unroll
-              for (int gi = 0; gi < 8; ++gi) {
-                const float smax =
-                    fmaxf(fmaxf(s[4 * gi], s[4 * gi + 1]), fmaxf(s[4 * gi + 2], s[4 * gi + 3]));
-                if (!(smax + kGumbelMax > gthr)) continue;
-                const uint32_t x4 = (uint32_t)(xq + 4 * gi);
-                const U4 o = philox10(U4{(x4 >> 2) | ((uint32_t)mc.b << 18), mc.c1, mc.c2, a.offset},
-                                      (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
-                const uint32_t wds[4] = {o.x, o.y, o.z, o.w};
+              for (int i = 0; i < 32; ++i) {
+                const float z = acc[i] + bias[i];
+                sv[i] = i < nv ? (STOCH ? __fdiv_rn(z, temp) : z) : -INFINITY;
+              }
+              float mx[16];
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                  const int i = 4 * gi + jj;
-                  if (i >= nv) continue;
-                  const float gk = s[i] + (-logf(-logf(u23(wds[jj]))));
-                  if (gk > gthr) {
-                    topk_insert<KMAX>(L2, I2, gk, xq + i);
-                    gthr = kth<KMAX>(L2, k);
+              for (int i = 0; i < 16; ++i) mx[i] = fmaxf(sv[i], sv[i + 16]);
+#pragma unroll
+              for (int w = 8; w; w >>= 1)
+#pragma unroll
+                for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+              const float mt = mx[0];
+              float ex[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ex[i] = ex2_approx((sv[i] - mt) * kLog2e);
+#pragma unroll
+              for (int w = 16; w; w >>= 1)
+#pragma unroll
+                for (int i = 0; i < w; ++i) ex[i] += ex[i + w];
+              const float st = ex[0];
+              if (mt > m) {
+                ssum = ssum * ex2_approx((m - mt) * kLog2e) + st;
+                m = mt;
+              } else {
+                ssum += st * ex2_approx((mt - m) * kLog2e);
+              }
+              if constexpr (STOCH) {
+                // Gumbel keys; four consecutive tokens share one Philox counter
+                if (mt + kGumbelMax > gthr) {
+#pragma unroll
+                  for (int gi = 0; gi < 8; ++gi) {
+                    const float smax = fmaxf(fmaxf(sv[4 * gi], sv[4 * gi + 1]),
+                                             fmaxf(sv[4 * gi + 2], sv[4 * gi + 3]));
+                    if (!(smax + kGumbelMax > gthr)) continue;
+                    const uint32_t x4 = (uint32_t)(xq + 4 * gi);
+                    const U4 o =
+                        philox10(U4{(x4 >> 2) | ((uint32_t)mc.b << 18), mc.c1, mc.c2, a.offset},
+                                 (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
+                    const uint32_t wds[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                      const int i = 4 * gi + jj;
+                      if (i >= nv) continue;
+                      const float gk = sv[i] + (-logf(-logf(u23(wds[jj]))));
+                      if (gk > gthr) {
+                        topk_insert<KMAX>(L2, I2, gk, xq + i);
+                        gthr = kth<KMAX>(L2, k);
+                      }
+                    }
                   }
+                }
+              }
+              // top-k of s: while the block's best left beats the k-th best so
+              // far (at most k rounds), insert it (lowest token among equal
+              // values first) and take it out of the block
+              if (mt > thr) {
+                float bm = mt;
+#pragma unroll 1
+                for (int rd = 0; rd < k && bm > thr; ++rd) {
+                  uint32_t eq = 0;
+#pragma unroll
+                  for (int i = 0; i < 32; ++i) eq |= (sv[i] == bm ? 1u : 0u) << i;
+                  const int ix = __ffs(eq) - 1;
+                  topk_insert<KMAX>(L1, I1, bm, xq + ix);
+                  thr = kth<KMAX>(L1, k);
+#pragma unroll
+                  for (int i = 0; i < 32; ++i) sv[i] = (i == ix) ? -INFINITY : sv[i];
+#pragma unroll
+                  for (int i = 0; i < 16; ++i) mx[i] = fmaxf(sv[i], sv[i + 16]);
+#pragma unroll
+                  for (int w = 8; w; w >>= 1)
+#pragma unroll
+                    for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+                  bm = mx[0];
                 }
               }
             }
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[ab]);
+          ++e_tile;
         }
-        // this quadrant's partials of the owned column, then one thread per
-        // column merges the four quadrants into the CTA's partial
-        named_bar(2, S::kEpiWarps * 32);
-        float* ql1v = tbuf;  // [4][NT][KMAX]
-        int32_t* ql1i = (int32_t*)(ql1v + 4 * NT * KMAX);
-        float* ql2v = (float*)(ql1i + 4 * NT * KMAX);
-        int32_t* ql2i = (int32_t*)(ql2v + (STOCH ? 4 * NT * KMAX : 0));
-        float2* qst = (float2*)(ql2i + (STOCH ? 4 * NT * KMAX : 0));  // [4][NT]
+        // every part's partial of every node into the exchange, then one
+        // thread per node merges them into the CTA's partial of the node
+        constexpr int kEx = 2 + 2 * KMAX * (STOCH ? 2 : 1);  // words per (part, node)
         {
-          const int col = eg * 32 + lane;
-          qst[q * NT + col] = make_float2(m, ssum);
+          float* mine = exch + ((size_t)part * NT + c) * kEx;
+          mine[0] = m;
+          mine[1] = ssum;
 #pragma unroll
           for (int i = 0; i < KMAX; ++i) {
-            ql1v[(q * NT + col) * KMAX + i] = L1[i];
-            ql1i[(q * NT + col) * KMAX + i] = I1[i];
+            mine[2 + i] = L1[i];
+            mine[2 + KMAX + i] = __int_as_float(I1[i]);
             if (STOCH) {
-              ql2v[(q * NT + col) * KMAX + i] = L2[i];
-              ql2i[(q * NT + col) * KMAX + i] = I2[i];
+              mine[2 + 2 * KMAX + i] = L2[i];
+              mine[2 + 3 * KMAX + i] = __int_as_float(I2[i]);
             }
           }
         }
         named_bar(2, S::kEpiWarps * 32);
-        const int par = wave & 1;
-        for (int c = threadIdx.x - 64; c < NT; c += S::kEpiWarps * 32) {
-          if (!meta[c].valid) continue;
+        const int cn = threadIdx.x;  // node merged by this thread
+        if (cn < NT && meta[cn].valid) {
+          const int par = wave & 1;
           float mx = -INFINITY;
-          for (int qq = 0; qq < 4; ++qq) mx = fmaxf(mx, qst[qq * NT + c].x);
+          for (int pp = 0; pp < S::kParts; ++pp)
+            mx = fmaxf(mx, exch[((size_t)pp * NT + cn) * kEx]);
           float sv = 0.f;
           if (mx != -INFINITY)
-            for (int qq = 0; qq < 4; ++qq) {
-              const float2 rv = qst[qq * NT + c];
-              if (rv.x != -INFINITY) sv += rv.y * exp2f((rv.x - mx) * kLog2e);
+            for (int pp = 0; pp < S::kParts; ++pp) {
+              const float* e = exch + ((size_t)pp * NT + cn) * kEx;
+              if (e[0] != -INFINITY) sv += e[1] * exp2f((e[0] - mx) * kLog2e);
             }
-          a.pstats[par][(size_t)c * ncta + cx] = make_float2(mx, sv);
+          a.pstats[par][(size_t)cn * ncta + cx] = make_float2(mx, sv);
           for (int lst = 0; lst < (STOCH ? 2 : 1); ++lst) {
-            const float* LV = lst ? ql2v : ql1v;
-            const int32_t* LI = lst ? ql2i : ql1i;
-            float* OV = (lst ? a.pgv[par] : a.plv[par]) + (size_t)c * k * ncta + cx;
-            int32_t* OI = (lst ? a.pgi[par] : a.pli[par]) + (size_t)c * k * ncta + cx;
-            int h[4] = {0, 0, 0, 0};  // heads of the four quadrant lists
+            float* OV = (lst ? a.pgv[par] : a.plv[par]) + (size_t)cn * k * ncta + cx;
+            int32_t* OI = (lst ? a.pgi[par] : a.pli[par]) + (size_t)cn * k * ncta + cx;
+            const int off = 2 + (lst ? 2 * KMAX : 0);
+            int hd[S::kParts];  // heads of the parts' sorted lists
+#pragma unroll
+            for (int pp = 0; pp < S::kParts; ++pp) hd[pp] = 0;
             for (int i = 0; i < k; ++i) {
-              int bw = -1;
+              int bw = 0;
               float bv = -INFINITY;
               int32_t bi = 0x7fffffff;
-              for (int w = 0; w < 4; ++w) {
-                if (h[w] >= k) continue;
-                const float v = LV[(w * NT + c) * KMAX + h[w]];
-                const int32_t id = LI[(w * NT + c) * KMAX + h[w]];
-                if (bw < 0 || ranks_first(v, id, bv, bi)) {
-                  bw = w;
+              bool have = false;
+#pragma unroll
+              for (int pp = 0; pp < S::kParts; ++pp) {
+                if (hd[pp] >= k) continue;
+                const float* e = exch + ((size_t)pp * NT + cn) * kEx + off;
+                const float v = e[hd[pp]];
+                const int32_t id = __float_as_int(e[KMAX + hd[pp]]);
+                if (!have || ranks_first(v, id, bv, bi)) {
+                  have = true;
+                  bw = pp;
                   bv = v;
                   bi = id;
                 }
               }
-              ++h[bw];
+#pragma unroll
+              for (int pp = 0; pp < S::kParts; ++pp) hd[pp] += (pp == bw) ? 1 : 0;
               OV[(size_t)i * ncta] = bv;
               OI[(size_t)i * ncta] = bi;
             }
@@ -913,35 +1014,54 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
       // ---- every CTA's partials of this wave are written: meet, bounded
       if (ct == 0) {
         const bool arrive = !(wave == 0 && cx == a.stall_cta);
-        if (!*abort_flag) grid_sync(a, (unsigned)wave, arrive, abort_flag);
+        if (!*abort_flag) grid_sync(a, 2u * wave, arrive, abort_flag);
         if (*abort_flag) atomicExch(a.grid_abort, 1);
         misc[6] = *abort_flag;
         misc[1] = 0;
       }
       named_bar(1, NCT);
       if (misc[6]) break;
-      // ---- merge every node's partials (one warp per node): its log-sum-exp
+      // ---- merge: node row e is merged by one warp of CTA e % ncta, which
+      // alone reads the row's ncta partials (148 CTAs reading the same lines
+      // at once would queue on the same L2 slices).  Per row: its log-sum-exp
       // and the kb best values of s with their tokens (T = 0) or the tokens
-      // of its Gumbel sample (T > 0)
+      // of its Gumbel sample (T > 0), into the merged-row buffer.
       {
         const int par = wave & 1;
-        const int cw = warp - 1;
-        for (int e = cw; e < n_rows; e += S::kCWarps) {
+        for (int e = cx + cw * ncta; cw < S::kMergeWarps && e < n_rows;
+             e += ncta * S::kMergeWarps) {
           const Row rw = rows[e];
           const int kb = reqs[rw.b].kb;
           const size_t prow = (size_t)e * ncta;
           const float lse = merge_node<KMAX>(
               a.pstats[par] + prow, a.plv[par] + prow * k, a.pli[par] + prow * k,
               STOCH ? a.pgv[par] + prow * k : nullptr, STOCH ? a.pgi[par] + prow * k : nullptr,
-              ncta, k, kb, lane, r_lq + e * k, STOCH ? nullptr : r_tok + e * k,
-              STOCH ? r_tok + e * k : nullptr, msv + cw * 32, msi + cw * 32);
-          __syncwarp();
-          if (lane == 0) r_lse[e] = lse;
-          for (int j = lane; j < kb; j += 32) r_lq[e * k + j] -= lse;
+              ncta, k, kb, lane, a.mrg_val + (size_t)e * k,
+              STOCH ? nullptr : a.mrg_tok + (size_t)e * k, STOCH ? a.mrg_tok + (size_t)e * k : nullptr,
+              msv + cw * 32, msi + cw * 32);
+          if (lane == 0) a.mrg_lse[e] = lse;
           __syncwarp();
         }
       }
       named_bar(1, NCT);
+      if (ct == 0) {
+        if (!*abort_flag) grid_sync(a, 2u * wave + 1, true, abort_flag);
+        if (*abort_flag) atomicExch(a.grid_abort, 1);
+        misc[6] = *abort_flag;
+      }
+      named_bar(1, NCT);
+      if (misc[6]) break;
+      // ---- every CTA reads the merged rows: log q of the kb best, tokens
+      for (int idx = ct; idx < n_rows * k; idx += NCT) {
+        const int e = idx / k, j = idx % k;
+        const float lse = __ldcg(a.mrg_lse + e);
+        r_lq[idx] = __ldcg(a.mrg_val + idx) - lse;
+        r_tok[idx] = __ldcg(a.mrg_tok + idx);
+        if (j == 0) r_lse[e] = lse;
+      }
+      named_bar(1, NCT);
+      // the weights of the next wave may stream while the selection runs
+      if (ct == 0) mbar_arrive(gate);
       // ---- best-first selection, request by request (the same in every CTA)
       for (int b = 0; b < a.batch; ++b)
         p_select<NCT>(a, b, reqs, lists, cands, sorted, keys, r_lse, r_lq, r_tok, rows,
@@ -953,6 +1073,11 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
     // the build is over (or was abandoned): the producer stops
     if (ct == 0) {
       *done_flag = 1;
+      // the producer may be suspended on the gate or on a ring slot that no
+      // MMA will free any more: complete those phases so that it wakes, sees
+      // the flag and stops (every MMA of the build has completed by now)
+      mbar_arrive(gate);
+      for (int st = 0; st < a.stages; ++st) mbar_arrive(&empty[st]);
       if (writer && STOCH && !misc[6]) *a.mat_count = misc[2];
       // The last CTA out resets the barrier words for the next launch on this
       // workspace: every CTA has left its last barrier wait by then.
@@ -964,9 +1089,8 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
         atomicExch(exits, 0u);
       }
     }
-    if (warp == 1 && lane == 0) {
+    if (warp == S::kWarpMma && lane == 0) {
       // every MMA this thread issued has completed before TMEM is released
-      uint64_t* drain = tempty + S::kAccBufs;
       tc_commit(drain);
       const uint64_t tw = globaltimer_ns();
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - tw < 50000000ull) {
@@ -974,26 +1098,32 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
     }
   }
   __syncthreads();
-  if (warp == 1) {
+  if (warp == S::kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem_base, S::kTmemCols);
   }
 }
 
+}  // namespace dt
+
+namespace dt {
+
 // ---------------------------------------------------------------- host side --
 int gemm_kmax(int k);
-bool gemm_can_gather(int r, int nt);
+bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows,
+                           uint32_t box_rows);
 
-// Node columns of a persistent build of this shape (every wave fits one
+// Node rows of a persistent build of this shape (every wave fits one MMA
 // tile of them), or 0 when the build runs as one launch pair per wave.
 int pbuild_cols(int batch, int Nmax, int r) {
   const long long m = (long long)batch * Nmax;
   const int nt = m <= 32 ? 32 : m <= 64 ? 64 : 0;
-  return (nt && gemm_can_gather(r, nt)) ? nt : 0;
+  return (nt && r <= 512) ? nt : 0;
 }
 
 template <int NG, bool STOCH, int KMAX>
-static cudaError_t pbuild_cfg(const CUtensorMap& tmW, PBuildArgs a, int ncta, cudaStream_t s) {
+static cudaError_t pbuild_cfg(const CUtensorMap& tmW, const CUtensorMap& tmW128, PBuildArgs a,
+                              int ncta, cudaStream_t s) {
   using S = PShape<NG>;
   auto kern = pbuild_kernel<NG, STOCH, KMAX>;
   const int esz = a.l_bf16 ? 2 : 4;
@@ -1001,15 +1131,15 @@ static cudaError_t pbuild_cfg(const CUtensorMap& tmW, PBuildArgs a, int ncta, cu
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return cudaErrorInvalidDevice;
-  // the deepest stage ring that fits next to everything else
-  int stages = 12;
+  // the deepest stage ring (32 KB stages) that fits next to everything else
+  int stages = 8;
   size_t bytes = 0;
-  for (; stages >= 4; --stages) {
+  for (; stages >= 2; --stages) {
     bytes = p_layout<NG>(stages, a.r, a.k, a.Nmax, a.batch, a.Bk, a.span, esz, KMAX, STOCH).total +
             1024;
     if (bytes <= (size_t)optin) break;
   }
-  if (stages < 4) return cudaErrorNotSupported;
+  if (stages < 2) return cudaErrorNotSupported;
   a.stages = stages;
   cudaError_t e = ensure_smem(kern, bytes);
   if (e != cudaSuccess) return e;
@@ -1029,23 +1159,28 @@ static cudaError_t pbuild_cfg(const CUtensorMap& tmW, PBuildArgs a, int ncta, cu
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tmW, a);
+  e = cudaLaunchKernelEx(&cfg, kern, tmW, tmW128, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 // One cooperative launch for the whole build (see the top of this file).
 // Returns cudaErrorNotSupported, with nothing enqueued, when the shape does
-// not fit it.
-cudaError_t launch_pbuild(const CUtensorMap& tmW, PBuildArgs a, int ncta, cudaStream_t s) {
+// not fit it.  Bm [V][r] bf16 is streamed in tiles of 256 (and 128) rows.
+cudaError_t launch_pbuild(const uint16_t* d_markov_b, PBuildArgs a, int ncta, cudaStream_t s) {
   const int nt = pbuild_cols(a.batch, a.Nmax, a.r);
   if (!nt || ncta < 1) return cudaErrorNotSupported;
+  CUtensorMap tmW, tmW128;
+  if (!make_tmap_bf16_kmajor(&tmW, d_markov_b, a.r, a.V, 256) ||
+      !make_tmap_bf16_kmajor(&tmW128, d_markov_b, a.r, a.V, 128))
+    return cudaErrorInvalidValue;
   a.span = ((a.n_vtiles + ncta - 1) / ncta) * kTileV;
   a.cap = a.Nmax + a.Nmax * a.k;
   const bool st = a.temp > 0.f;
   const int km = gemm_kmax(a.k);
-#define DT_PB_CASE(NG, ST, KM) \
-  if (nt == 32 * NG && st == ST && km == KM) return pbuild_cfg<NG, ST, KM>(tmW, a, ncta, s);
+#define DT_PB_CASE(NG, ST, KM)                  \
+  if (nt == 32 * NG && st == ST && km == KM) \
+    return pbuild_cfg<NG, ST, KM>(tmW, tmW128, a, ncta, s);
   DT_PB_CASE(1, false, 4)
   DT_PB_CASE(1, false, 16)
   DT_PB_CASE(1, true, 4)
