@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdtree.so")
 SOURCES = ["api_build.cu", "markov_gemm.cu", "frontier.cu", "accept.cu", "verify_attn.cu",
-           "treeflash.cu", "accept_noalloc.cu", "load_policy.cu", "pbuild.cu",
+           "treeflash.cu", "attn_tc.cu", "accept_noalloc.cu", "load_policy.cu", "pbuild.cu",
            "calibration.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

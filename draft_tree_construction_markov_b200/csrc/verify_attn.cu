@@ -13,7 +13,9 @@
 // accumulation and an online softmax; the ancestor bitmask is applied only to
 // the tree columns.  A combine kernel merges the splits.  fp32 inputs use a
 // plain per-(row, head) kernel.
-#include "common.cuh"
+#include <algorithm>
+
+#include "attn_tc.cuh"
 
 namespace dt {
 
@@ -436,6 +438,22 @@ struct AttnPlan {
   size_t part_o_bytes, part_ml_bytes;
 };
 
+// The tensor-core kernel (attn_tc.cu): 128-column splits, one partial row per
+// (tree row, query head) of each KV head.
+static AttnPlan attn_tc_plan(int batch, int Nmax, int Hq, int Hkv, int d, int max_prefix) {
+  AttnPlan p;
+  const int G = Hq / Hkv;
+  p.n_rblocks = 1;
+  p.rows_per_cta = p.rpad = G * (Nmax + 1);
+  p.warps = 4;
+  p.cols_per_split = 128;
+  p.splits = (max_prefix + Nmax + 1 + 127) / 128;
+  const size_t rows = (size_t)p.splits * batch * Hkv * p.rpad;
+  p.part_o_bytes = rows * d * 4;
+  p.part_ml_bytes = rows * 8;
+  return p;
+}
+
 static AttnPlan attn_plan(int batch, int Nmax, int Hq, int Hkv, int d, int max_prefix) {
   AttnPlan p;
   const int G = Hq / Hkv;
@@ -470,7 +488,10 @@ size_t dt_tree_verify_attn_workspace_bytes(int batch, int Nmax, int Hq, int Hkv,
   if (batch <= 0 || Nmax <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || d <= 0 || max_prefix < 0)
     return 0;
   AttnPlan p = attn_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
-  return kWsHeader + ((p.part_ml_bytes + 255) & ~(size_t)255) + p.part_o_bytes + 256;
+  AttnPlan t = attn_tc_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
+  const size_t ml = std::max(p.part_ml_bytes, t.part_ml_bytes);
+  const size_t o = std::max(p.part_o_bytes, t.part_o_bytes);
+  return kWsHeader + ((ml + 255) & ~(size_t)255) + o + 256;
 }
 
 dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const void* d_v_prefix,
@@ -490,7 +511,10 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const voi
   const size_t need = dt_tree_verify_attn_workspace_bytes(batch, Nmax, Hq, Hkv, d, max_prefix);
   if (!ws || ws_bytes < need) return DT_EWORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
-  AttnPlan p = attn_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
+  // bf16: the tensor-core kernel; fp32 inputs: the plain per-(row, head) kernel
+  const bool tc = dt == DT_BF16;
+  AttnPlan p = tc ? attn_tc_plan(batch, Nmax, Hq, Hkv, d, max_prefix)
+                  : attn_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
   AttnArgs a;
   a.q = d_q;
   a.kp = d_k_prefix;
@@ -516,8 +540,12 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const voi
   a.rpad = p.rpad;
   uint8_t* w = (uint8_t*)ws;
   a.status = (int32_t*)w;
-  a.part_ml = (float2*)(w + kWsHeader);
-  a.part_o = (float*)(w + kWsHeader + ((p.part_ml_bytes + 255) & ~(size_t)255));
+  {
+    AttnPlan p0 = attn_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
+    const size_t ml = std::max(p0.part_ml_bytes, p.part_ml_bytes);
+    a.part_ml = (float2*)(w + kWsHeader);
+    a.part_o = (float*)(w + kWsHeader + ((ml + 255) & ~(size_t)255));
+  }
   a.out = d_out;
   a.out_bf16 = dt == DT_BF16;
   if (cudaMemsetAsync(a.status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
@@ -531,21 +559,34 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const voi
     attn_f32_kernel<<<dim3(batch * (Nmax + 1), Hq), 128, smem, s>>>(a, max_cols);
     return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ECUDA;
   }
-  const size_t smem = ((size_t)p.rows_per_cta + 4 * kChunk) * (d + 8) * 2;
-  dim3 grid(p.splits, Hkv, batch * p.n_rblocks);
-  const int threads = 32 * std::max(p.warps, 4);
   {
-  ProfileScope ps(DT_K_ATTN, s);
-  if (d == 128) {
-    if (ensure_smem(attn_bf16_kernel<128>, smem) != cudaSuccess)
-      return DT_ECUDA;
-    attn_bf16_kernel<128><<<grid, threads, smem, s>>>(a);
-  } else {
-    if (ensure_smem(attn_bf16_kernel<64>, smem) != cudaSuccess)
-      return DT_ECUDA;
-    attn_bf16_kernel<64><<<grid, threads, smem, s>>>(a);
-  }
-  if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+    AttnTcArgs t;
+    t.q = (const uint16_t*)d_q;
+    t.kp = (const uint16_t*)d_k_prefix;
+    t.vp = (const uint16_t*)d_v_prefix;
+    t.pstart = d_prefix_start;
+    t.plen = d_prefix_len;
+    t.kt = (const uint16_t*)d_k_tree;
+    t.vt = (const uint16_t*)d_v_tree;
+    t.anc = d_anc;
+    t.n_nodes = d_n_nodes;
+    t.batch = batch;
+    t.Nmax = Nmax;
+    t.Hq = Hq;
+    t.Hkv = Hkv;
+    t.d = d;
+    t.G = Hq / Hkv;
+    t.max_prefix = max_prefix;
+    t.heads_per_cta = attn_tc_heads_per_cta(t.G, Nmax);
+    t.n_groups = t.G / t.heads_per_cta;
+    t.scale_log2 = scale * kAttnL2e;
+    t.part_o = a.part_o;
+    t.part_ml = a.part_ml;
+    t.splits = p.splits;
+    t.rpad = p.rpad;
+    t.status = a.status;
+    ProfileScope ps(DT_K_ATTN, s);
+    if (launch_attn_tc(t, s) != cudaSuccess) return DT_ECUDA;
   }
   ProfileScope ps(DT_K_ATTN_COMBINE, s);
   const int items = batch * (Nmax + 1) * Hq;

@@ -137,7 +137,7 @@ class Workload:
     philox_offset: int = 0
 
 
-def _block_logits(g, Bk, V, scale, plant, dtype):
+def _block_logits(g, Bk, V, scale, plant, dtype, dyadic=True):
     L = (scale * g.standard_normal((Bk, V))).astype(np.float32)
     planted = g.integers(0, V, size=Bk)
     kind, m0, m1 = plant
@@ -149,26 +149,36 @@ def _block_logits(g, Bk, V, scale, plant, dtype):
             others = np.delete(L[d], planted[d])
             L[d, planted[d]] = np.float32(others.max() + m)
     if dtype == "bf16":
-        L = _dyadic(bf16_round(L), 14)
+        L = _dyadic(bf16_round(L), 14) if dyadic else bf16_round(L)
     else:
-        L = _dyadic(L, 10)
+        L = _dyadic(L, 10) if dyadic else L
     return L
 
 
-def make_workload(name: str, seed: int = 0, **over) -> Workload:
-    """Draw the inputs of one round of configuration ``name`` (sizes overridable)."""
+def make_workload(name: str, seed: int = 0, dyadic: bool = True, **over) -> Workload:
+    """Draw the inputs of one round of configuration ``name`` (sizes overridable).
+
+    ``dyadic=False`` keeps the Markov factors and block logits as plain bf16
+    values (no snapping to the dyadic grids): the drafter logits are then no
+    longer exact in fp32, and integer decisions must be compared only where
+    their margins are well above fp32 rounding.
+    """
     c = dict(CONFIGS[name])
     c.update(over)
     V, Bk, r, batch = c["V"], c["Bk"], c["r"], c["batch"]
     g = rng(seed, _T_MARKOV)
     sab = c["sigma_ab"]
-    A = _dyadic(np.clip(sab * g.standard_normal((V, r)), -1.5, 1.5), 7)
-    Bt = _dyadic(np.clip(sab * g.standard_normal((V, r)), -1.5, 1.5), 7)
+    if dyadic:
+        A = _dyadic(np.clip(sab * g.standard_normal((V, r)), -1.5, 1.5), 7)
+        Bt = _dyadic(np.clip(sab * g.standard_normal((V, r)), -1.5, 1.5), 7)
+    else:
+        A = bf16_round((sab * g.standard_normal((V, r))).astype(np.float32))
+        Bt = bf16_round((sab * g.standard_normal((V, r))).astype(np.float32))
     L = np.empty((batch, Bk, V), np.float32)
     Lt = np.empty((batch, Bk + 1, V), np.float32)
     for b in range(batch):
         gb = rng(seed, _T_BLOCK, b)
-        L[b] = _block_logits(gb, Bk, V, c["L_scale"], c["plant"], c["logit_dtype"])
+        L[b] = _block_logits(gb, Bk, V, c["L_scale"], c["plant"], c["logit_dtype"], dyadic)
         Lt[b, :Bk] = L[b]
         extra = (c["L_scale"] * gb.standard_normal(V)).astype(np.float32)
         Lt[b, Bk] = _dyadic(bf16_round(extra), 14) if c["logit_dtype"] == "bf16" else _dyadic(extra, 10)

@@ -70,20 +70,28 @@ def ar_approximator(h, e_prev, w_norm_h, w_norm_e, W_gate, W_up, W_down, store=N
 
 
 def stage1_sets(h, W_lm, M):
-    """S_i (i = 1..gamma): the M best tokens of W_lm h_i; returns list of arrays."""
+    """S_i (i = 1..gamma): the M best tokens of W_lm h_i; returns list of arrays
+    (the gamma matrix-vector products as one matrix product W_lm [h_1 ... h_gamma])."""
     W = np.asarray(W_lm, np.float64)
-    return [top_k_desc(W @ np.asarray(h[i], np.float64), M) for i in range(len(h))]
+    Z = W @ np.asarray(h, np.float64).T
+    return [top_k_desc(Z[:, i], M) for i in range(len(h))]
 
 
 def stage2_distributions(h, E, root, sets, w_norm_h, w_norm_e, W_gate, W_up, W_down, W_lm,
                          store=None):
-    """{(depth, prev): (s, lse)} for depth 1 (prev = root) and every prev in S_{depth-1}."""
+    """{(depth, prev): (s, lse)} for depth 1 (prev = root) and every prev in S_{depth-1}.
+
+    The LM head of every evaluation is one column of a single matrix product
+    W_lm [h'_1 ... h'_n] (the same dot products as one matrix-vector product
+    per evaluation, read with one pass over W_lm)."""
     W = np.asarray(W_lm, np.float64)
     out = {}
     evals = [(1, int(root))] + [(i, int(t)) for i in range(2, len(h) + 1) for t in sets[i - 2]]
-    for d, prev in evals:
-        hp = ar_approximator(h[d - 1], E[prev], w_norm_h, w_norm_e, W_gate, W_up, W_down, store)
-        out[(d, prev)] = scaled_logits(W @ hp, 0.0)
+    H = np.stack([ar_approximator(h[d - 1], E[prev], w_norm_h, w_norm_e, W_gate, W_up, W_down,
+                                  store) for d, prev in evals], axis=1)
+    Z = W @ H
+    for j, (d, prev) in enumerate(evals):
+        out[(d, prev)] = scaled_logits(Z[:, j], 0.0)
     return out
 
 
