@@ -5,13 +5,14 @@
 // section (siblings sampled without replacement, residuals matched in
 // recursive rejection); PCTree summary, "setup" (greedy verification).
 //
-// Two launches.  A pre-pass over every target row of every request (row 0 =
-// root, row i+1 = node i, rows past n_nodes skipped) computes, per row chunk,
-// the argmax (T = 0) or the max and sum of exp(t / T) (T > 0).  The walk then
-// runs one warp per request at T = 0, where it only compares child tokens
-// with row argmaxes, and one thread-block cluster per request at T > 0, where
-// every rejected sibling costs one vocabulary-wide residual pass,
-// r <- max(p - q_j, 0), split over the cluster's CTAs.
+// A pre-pass over every target row of every request (row 0 = root, row i+1 =
+// node i, rows past n_nodes skipped) computes, per row chunk, the argmax
+// (T = 0) or the max and sum of exp(t / T) (T > 0).  At T = 0 that is the
+// only launch: the last pre-pass CTA of a request (an arrival counter per
+// request) walks the tree with one warp, comparing child tokens with row
+// argmaxes.  At T > 0 a second launch walks each request on one thread-block
+// cluster, where every rejected sibling costs one vocabulary-wide residual
+// pass, r <- max(p - q_j, 0), split over the cluster's CTAs.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -36,14 +37,11 @@ struct AccParts {
   float* ps;    // [rows_total][splits] sum exp(t/T - max)   (T > 0)
 };
 
-// Pre-pass: grid (splits, batch * (Nmax + 1)).
+// Partial statistics of chunk blockIdx.x of target row row_g (all threads of
+// the CTA): argmax (T = 0) or (max, sum exp(t / T - max)) (T > 0).
 template <bool STOCH>
-__global__ void __launch_bounds__(kPreThreads)
-    accept_prepass_kernel(const void* t, int tbf16, const int32_t* n_nodes, int Nmax, int V,
-                          int splits, float temp, AccParts parts) {
-  const int row_g = blockIdx.y;
-  const int b = row_g / (Nmax + 1), row = row_g % (Nmax + 1);
-  if (row > min(n_nodes[b], Nmax)) return;
+__device__ __forceinline__ void prepass_chunk(const void* t, int tbf16, int row_g, int V,
+                                              int splits, float temp, AccParts parts) {
   const int chunk = ((V + splits - 1) / splits + 7) & ~7;
   const int x0 = blockIdx.x * chunk, x1 = min(V, x0 + chunk);
   const size_t base = (size_t)row_g * V;
@@ -147,6 +145,17 @@ __global__ void __launch_bounds__(kPreThreads)
   }
 }
 
+// Pre-pass: grid (splits, batch * (Nmax + 1)).
+template <bool STOCH>
+__global__ void __launch_bounds__(kPreThreads)
+    accept_prepass_kernel(const void* t, int tbf16, const int32_t* n_nodes, int Nmax, int V,
+                          int splits, float temp, AccParts parts) {
+  const int row_g = blockIdx.y;
+  const int b = row_g / (Nmax + 1), row = row_g % (Nmax + 1);
+  if (row > min(n_nodes[b], Nmax)) return;
+  prepass_chunk<STOCH>(t, tbf16, row_g, V, splits, temp, parts);
+}
+
 struct WalkArgs {
   const void* t;
   int tbf16;
@@ -167,30 +176,39 @@ struct WalkArgs {
   int32_t* status;
 };
 
-// Greedy walk: one warp per request; the tree is staged in shared memory and
-// each visited row's split partials are combined lane-parallel.
-__global__ void greedy_walk_kernel(WalkArgs w) {
-  const int b = blockIdx.x, lane = threadIdx.x;
-  __shared__ int32_t s_tok[64], s_par[64];
-  int n = w.n_nodes[b];
-  if (n < 0 || n > w.Nmax) {
-    if (lane == 0) set_status(w.status, DT_EDEVICE);
-    n = n < 0 ? 0 : w.Nmax;
+// T = 0 in one launch: grid (splits, batch * (Nmax + 1)); each CTA the argmax
+// of one chunk of one target row; the last CTA of a request to finish walks
+// its tree: one warp per row merges the row's split partials, then one warp
+// follows the argmax tokens down the tree in shared memory.  counters [batch]
+// start at zero and are left at zero.
+__global__ void __launch_bounds__(kPreThreads)
+    accept_greedy_kernel(WalkArgs w, int32_t* counters) {
+  const int row_g = blockIdx.y;
+  const int b = row_g / (w.Nmax + 1), row = row_g % (w.Nmax + 1);
+  const int n_raw = w.n_nodes[b];
+  const int n = min(max(n_raw, 0), w.Nmax);
+  if (row > n) return;  // uniform; rows past the tree are not counted
+  prepass_chunk<false>(w.t, w.tbf16, row_g, w.V, w.splits, 0.f, w.parts);
+  __shared__ int s_last;
+  __shared__ int32_t s_tok[64], s_par[64], s_arg[65];
+  if (threadIdx.x == 0) {
+    __threadfence();  // this CTA's partial before its arrival
+    const int total = w.splits * (n + 1);
+    s_last = atomicAdd(&counters[b], 1) == total - 1;
+    if (s_last) counters[b] = 0;  // every CTA of the request has arrived
   }
-  for (int i = lane; i < n; i += 32) {
-    s_tok[i] = w.tokens[(size_t)b * w.Nmax + i];
-    s_par[i] = w.parents[(size_t)b * w.Nmax + i];
-  }
-  __syncwarp();
-  int node = -1, nacc = 0;
-  int32_t a = 0;
-  while (true) {
-    const size_t rg = (size_t)b * (w.Nmax + 1) + (node + 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0 && (n_raw < 0 || n_raw > w.Nmax)) set_status(w.status, DT_EDEVICE);
+  for (int r = warp; r <= n; r += kPreThreads / 32) {
+    const size_t rg = (size_t)b * (w.Nmax + 1) + r;
     float best = -INFINITY;
     int32_t bi = 0x7fffffff;
     for (int s = lane; s < w.splits; s += 32) {
-      const float v = w.parts.pv[rg * w.splits + s];
-      const int32_t id = w.parts.pi[rg * w.splits + s];
+      const float v = __ldcg(w.parts.pv + rg * w.splits + s);
+      const int32_t id = __ldcg(w.parts.pi + rg * w.splits + s);
       if (v > best || (v == best && id < bi)) {
         best = v;
         bi = id;
@@ -205,7 +223,18 @@ __global__ void greedy_walk_kernel(WalkArgs w) {
         bi = oi;
       }
     }
-    a = bi;
+    if (lane == 0) s_arg[r] = bi;
+  }
+  for (int i = threadIdx.x; i < n; i += kPreThreads) {
+    s_tok[i] = w.tokens[(size_t)b * w.Nmax + i];
+    s_par[i] = w.parents[(size_t)b * w.Nmax + i];
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  int node = -1, nacc = 0;
+  int32_t a = 0;
+  while (true) {
+    a = s_arg[node + 1];
     // children of `node` carry distinct tokens: at most one matches
     int next = -1;
     for (int i0 = 0; i0 < n; i0 += 32) {
@@ -486,7 +515,7 @@ size_t dt_tree_accept_workspace_bytes(int batch, int Nmax, int V) {
   if (batch <= 0 || Nmax <= 0 || V <= 0) return 0;
   const int rows = batch * (Nmax + 1);
   const int sp = accept_splits(rows, V);
-  size_t b = kWsHeader;
+  size_t b = kWsHeader + align256((size_t)batch * 4);  // status word, T = 0 arrival counters
   b += align256((size_t)rows * sp * 4) * 3;
   b += align256((size_t)batch * 2 * V * 4);
   return b;
@@ -511,6 +540,8 @@ dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt, const dt_tre
   uint8_t* p = (uint8_t*)ws;
   int32_t* status = (int32_t*)p;
   p += kWsHeader;
+  int32_t* counters = (int32_t*)p;
+  p += align256((size_t)batch * 4);
   AccParts parts;
   parts.pv = (float*)p;
   p += align256((size_t)rows * sp * 4);
@@ -519,19 +550,15 @@ dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt, const dt_tre
   parts.ps = (float*)p;
   p += align256((size_t)rows * sp * 4);
   float* rbuf = (float*)p;
-  if (cudaMemsetAsync(status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
+  // the status word and the arrival counters, which sit right after it
+  if (cudaMemsetAsync(status, 0, kWsHeader + (size_t)batch * 4, s) != cudaSuccess) return DT_ECUDA;
   dim3 grid(sp, rows);
   const int tb = tdt == DT_BF16;
-  {
-  ProfileScope ps(DT_K_ACCEPT_PREPASS, s);
-  if (temp > 0.f)
+  if (temp > 0.f) {
+    ProfileScope ps(DT_K_ACCEPT_PREPASS, s);
     accept_prepass_kernel<true><<<grid, kPreThreads, 0, s>>>(d_target_logits, tb, tree->d_n_nodes,
                                                              Nmax, V, sp, temp, parts);
-  else
-    accept_prepass_kernel<false><<<grid, kPreThreads, 0, s>>>(d_target_logits, tb,
-                                                              tree->d_n_nodes, Nmax, V, sp, temp,
-                                                              parts);
-  if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
+    if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
   }
   WalkArgs w;
   w.t = d_target_logits;
@@ -574,7 +601,8 @@ dt_status dt_tree_accept(const void* d_target_logits, dt_dtype tdt, const dt_tre
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, stoch_walk_kernel, w) != cudaSuccess) return DT_ECUDA;
   } else {
-    greedy_walk_kernel<<<batch, 32, 0, s>>>(w);
+    // pre-pass and walk in one launch
+    accept_greedy_kernel<<<grid, kPreThreads, 0, s>>>(w, counters);
   }
   if (cudaGetLastError() != cudaSuccess) return DT_ECUDA;
   return DT_OK;

@@ -52,7 +52,8 @@ extern "C" dt_status dt_tree_accept_noalloc(const void* d_target_logits, dt_dtyp
   if (need == 0 || need > kNoAllocScratchBytes) return DT_EUNSUPPORTED;  // beyond the fixed scratch
   void* ws = scratch_address();
   if (!ws) return DT_ECUDA;
-  // dt_tree_accept clears the status word itself; nothing else must start at zero
+  // dt_tree_accept clears the status word and its arrival counters itself;
+  // nothing else in the scratch must start at zero
   return dt_tree_accept(d_target_logits, tdt, tree, batch, Bk, V, Nmax, temp, philox_seed,
                         philox_offset, d_acc_nodes, d_n_acc, d_bonus, ws, kNoAllocScratchBytes,
                         stream);

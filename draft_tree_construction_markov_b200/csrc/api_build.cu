@@ -339,7 +339,10 @@ static dt_status run_waves(FrontierArgs f, GemmArgs g, const BuildLayout& L,
                            const CUtensorMap& tmW,
                            const CUtensorMap& tmH, const CUtensorMap& tmHm, int batch, int Bk,
                            int Nmax, float* d_draft_q, cudaStream_t s) {
-  const bool fits = pbuild_cols(batch, Nmax, f.r) > 0;
+  // At T > 0 the draft-q GEMM after the build reads its node rows through Hm
+  // when r is too large to gather them in shared memory; only the per-wave
+  // frontier fills Hm, so those builds run as waves.
+  const bool fits = pbuild_cols(batch, Nmax, f.r) > 0 && (f.temp == 0.f || f.Hm == nullptr);
   if (g_build_path == DT_BUILD_PERSISTENT && !fits) return DT_EUNSUPPORTED;
   bool waves = g_build_path == DT_BUILD_WAVES || !fits;
   if (!waves) {

@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnTcArgs a) {
   const int P = min(max(a.plen[b], 0), a.max_prefix);
   const int C = P + n + 1;                     // key columns of this request
   const int c0 = split * kTcKeys;
+  pdl_launch_dependents();  // the split combine may be scheduled (it waits for us)
   if (c0 >= C) return;                         // uniform: nothing to attend to here
   const int64_t ps = a.pstart[b];
   const int hpc = a.heads_per_cta;
@@ -100,36 +101,70 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnTcArgs a) {
     const uint16_t* src = a.q + (((size_t)b * N1 + (ok ? i : 0)) * a.Hq + head) * D + kc * 64 + c * 8;
     cp16(smem_u32(sq + kc * kTile + sw128(m, c)), src, ok);
   }
-  // K and V: key j of the split is column c0 + j: prefix row, or tree row.
-  // Lanes take consecutive keys, so the transposed V stores of a warp land in
-  // consecutive 2-byte slots of one d row.
+  // K and V: key j of the split is column c0 + j: prefix row, or tree row
   for (int idx = tid; idx < kTcKeys * KC * 8; idx += kTcThreads) {
-    const int j = idx % kTcKeys, c = (idx / kTcKeys) & 7, kc = idx / (kTcKeys * 8);
+    const int c = idx & 7, j = (idx >> 3) % kTcKeys, kc = (idx >> 3) / kTcKeys;
     const int col = c0 + j;
     const bool ok = col < C;
     size_t off;
-    const uint16_t *kb, *vb;
+    const uint16_t* kb;
     if (col < P) {
       off = ((size_t)(ps + col) * a.Hkv + kvh) * D;
       kb = a.kp;
-      vb = a.vp;
     } else {
-      const int t = ok ? col - P : 0;
-      off = (((size_t)b * N1 + t) * a.Hkv + kvh) * D;
+      off = (((size_t)b * N1 + (ok ? col - P : 0)) * a.Hkv + kvh) * D;
       kb = a.kt;
-      vb = a.vt;
     }
     off += kc * 64 + c * 8;
     cp16(smem_u32(sk + kc * kTile + sw128(j, c)), kb + (ok ? off : 0), ok);
-    const uint4 v = ok ? *(const uint4*)(vb + off) : make_uint4(0, 0, 0, 0);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    // V[j][d] for d = 64 kc + 8 c + e  ->  V^T row d, key j (key half j >> 6)
+  }
+  // V^T: a thread takes keys 2 u, 2 u + 1 and 8 consecutive d, and stores the
+  // 8 key pairs (4 bytes each) into 8 rows of V^T; lanes take consecutive
+  // pairs, so a warp's stores fill 128 contiguous bytes of each row
+  // (all of a thread's loads are issued before its first store)
+  constexpr int kVItems = (kTcKeys / 2) * KC * 8 / kTcThreads;
+  uint32_t vw[kVItems][2][4];
+#pragma unroll
+  for (int it = 0; it < kVItems; ++it) {
+    const int idx = tid + it * kTcThreads;
+    const int u = idx % (kTcKeys / 2), c = (idx / (kTcKeys / 2)) & 7,
+              kc = idx / (kTcKeys / 2 * 8);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int col = c0 + 2 * u + h;
+      const bool ok = col < C;
+      size_t off;
+      const uint16_t* vb;
+      if (col < P) {
+        off = ((size_t)(ps + col) * a.Hkv + kvh) * D;
+        vb = a.vp;
+      } else {
+        off = (((size_t)b * N1 + (ok ? col - P : 0)) * a.Hkv + kvh) * D;
+        vb = a.vt;
+      }
+      off += kc * 64 + c * 8;
+      const uint4 v = ok ? *(const uint4*)(vb + off) : make_uint4(0, 0, 0, 0);
+      vw[it][h][0] = v.x;
+      vw[it][h][1] = v.y;
+      vw[it][h][2] = v.z;
+      vw[it][h][3] = v.w;
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < kVItems; ++it) {
+    const int idx = tid + it * kTcThreads;
+    const int u = idx % (kTcKeys / 2), c = (idx / (kTcKeys / 2)) & 7,
+              kc = idx / (kTcKeys / 2 * 8);
+    // V[j][d] for d = 64 kc + 8 c + e  ->  V^T row d, keys j = 2 u, 2 u + 1
+    const int j = 2 * u;
     uint8_t* vt = sv + (j >> 6) * (D * 128);
     const int jc = (j & 63) >> 3, jb = (j & 7) * 2;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int d = kc * 64 + c * 8 + e;
-      *(uint16_t*)(vt + sw128(d, jc) + jb) = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+      const uint32_t lo = (vw[it][0][e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+      const uint32_t hi = (vw[it][1][e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+      *(uint32_t*)(vt + sw128(d, jc) + jb) = lo | (hi << 16);
     }
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
@@ -164,24 +199,53 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnTcArgs a) {
   const uint64_t am = (row_ok && i >= 1) ? a.anc[(size_t)b * a.Nmax + (i - 1)] : 0ull;
   float s[kTcKeys];
   if (ok) {
+    uint32_t r[kTcKeys / 16][16];
 #pragma unroll
-    for (int c4 = 0; c4 < kTcKeys / 16; ++c4) {
-      float v[16];
-      tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(16 * c4), v);
+    for (int c4 = 0; c4 < kTcKeys / 16; ++c4)
+      tmem_ld16_nowait(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(16 * c4), r[c4]);
+    tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) s[16 * c4 + e] = v[e];
+    for (int c4 = 0; c4 < kTcKeys / 16; ++c4)
+#pragma unroll
+      for (int e = 0; e < 16; ++e) s[16 * c4 + e] = __uint_as_float(r[c4][e]);
+  }
+  // allowed columns of this row among the split's 128, as 4 words of bits:
+  // the prefix, the root's tree row, and the rows of the row's ancestors
+  // (tree row t = node t - 1: bit t of 1 | anc << 1)
+  uint32_t allow[kTcKeys / 32];
+  {
+    const uint64_t tlo = 1ull | (am << 1), thi = am >> 63;  // tree-row bits 0..64
+#pragma unroll
+    for (int wd = 0; wd < kTcKeys / 32; ++wd) {
+      const int base = c0 + 32 * wd;  // column of bit 0
+      const int npre = min(max(P - base, 0), 32);
+      uint32_t word = npre == 32 ? 0xffffffffu : ((1u << npre) - 1u);
+      // tree columns: bit k is column base + k = P + t with t = base - P + k
+      const int t0 = base - P;
+      uint32_t tb = 0;
+      if (t0 > -32 && t0 <= 64) {
+        // 32 bits of the tree mask from bit t0 (bits below 0 are prefix columns)
+        uint64_t lo, hi;
+        if (t0 >= 0) {
+          lo = t0 < 64 ? (tlo >> t0) | (t0 ? (thi << (64 - t0)) : 0ull) : thi >> (t0 - 64);
+          hi = 0;
+          tb = (uint32_t)lo;
+        } else {
+          tb = (uint32_t)(tlo << (-t0));
+        }
+        (void)hi;
+      }
+      // columns at or past C (and past the tree) are not keys
+      const int nval = min(max(C - base, 0), 32);
+      const uint32_t inb = nval == 32 ? 0xffffffffu : ((1u << nval) - 1u);
+      word = (word | (tb & ~word)) & inb;
+      allow[wd] = row_ok ? word : 0u;
     }
   }
   float mx = -INFINITY;
 #pragma unroll
   for (int j = 0; j < kTcKeys; ++j) {
-    const int col = c0 + j;
-    bool allow = row_ok && col < C;
-    if (col >= P) {
-      const int t = col - P;  // tree row: 0 = root, t = node t-1
-      allow = allow && (t == 0 || (i >= 1 && ((am >> (t - 1)) & 1ull)));
-    }
-    s[j] = allow ? s[j] * a.scale_log2 : -INFINITY;
+    s[j] = ((allow[j >> 5] >> (j & 31)) & 1u) ? s[j] * a.scale_log2 : -INFINITY;
     mx = fmaxf(mx, s[j]);
   }
   float l = 0.f;
@@ -191,7 +255,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnTcArgs a) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float x = s[8 * c8 + e];
-      p[e] = (x == -INFINITY) ? 0.f : exp2f(x - mx);
+      float y;
+      asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x - mx));  // 2^-inf = 0
+      p[e] = (x == -INFINITY) ? 0.f : y;
       l += p[e];
     }
     uint4 pk;
@@ -232,15 +298,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnTcArgs a) {
     const size_t prow = (((size_t)split * a.batch + b) * a.Hkv + kvh) * a.rpad + rho;
     if (row_ok) a.part_ml[prow] = make_float2(mx, l);
     float4* dst = (float4*)(a.part_o + prow * D);
+    uint32_t r[D / 16][16];
 #pragma unroll
-    for (int c4 = 0; c4 < D / 16; ++c4) {
-      float v[16];
-      tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + 128u + (uint32_t)(16 * c4), v);
-      if (row_ok) {
+    for (int c4 = 0; c4 < D / 16; ++c4)
+      tmem_ld16_nowait(tmem + ((uint32_t)(32 * warp) << 16) + 128u + (uint32_t)(16 * c4), r[c4]);
+    tmem_wait_ld();
+    if (row_ok) {
+#pragma unroll
+      for (int c4 = 0; c4 < D / 16; ++c4)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          dst[4 * c4 + e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-      }
+          dst[4 * c4 + e] =
+              make_float4(__uint_as_float(r[c4][4 * e]), __uint_as_float(r[c4][4 * e + 1]),
+                          __uint_as_float(r[c4][4 * e + 2]), __uint_as_float(r[c4][4 * e + 3]));
     }
   }
   tc_fence_before();

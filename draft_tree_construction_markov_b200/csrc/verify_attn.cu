@@ -292,6 +292,7 @@ constexpr int kCombineWarps = 4;
 // Merge the column splits: one warp per (request, row, head); lanes cover
 // head_dim in 4-float vectors.  grid (ceil(batch*(Nmax+1)*Hq / 4)), 128 threads.
 __global__ void attn_combine_kernel(AttnArgs a) {
+  pdl_wait();  // the attention kernel's partials (no-op without a programmatic launch)
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
   const int per_b = (a.Nmax + 1) * a.Hq;
@@ -590,7 +591,14 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const voi
   }
   ProfileScope ps(DT_K_ATTN_COMBINE, s);
   const int items = batch * (Nmax + 1) * Hq;
-  attn_combine_kernel<<<(items + kCombineWarps - 1) / kCombineWarps, 32 * kCombineWarps, 0, s>>>(a);
+  const dim3 cgrid((items + kCombineWarps - 1) / kCombineWarps);
+  if (tc) {
+    // launched while the attention kernel runs; it waits for its partials
+    if (launch_pdl(attn_combine_kernel, cgrid, dim3(32 * kCombineWarps), 0, s, a) != cudaSuccess)
+      return DT_ECUDA;
+  } else {
+    attn_combine_kernel<<<cgrid, 32 * kCombineWarps, 0, s>>>(a);
+  }
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ECUDA;
 }
 

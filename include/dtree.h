@@ -448,10 +448,11 @@ typedef enum {
  * expansion (TreeSpark article, "core idea"; the exact wave schedule is
  * described with dt_tree_build).  The result is the same either way; this is
  * a tuning and diagnostic switch, set per host thread.
- *   DT_BUILD_AUTO        one persistent launch when batch * Nmax <= 64 and
- *                        r <= 256 (and the device can hold one such CTA per
- *                        SM), otherwise one GEMM and one frontier launch per
- *                        wave (the default);
+ *   DT_BUILD_AUTO        one persistent launch when batch * Nmax <= 64,
+ *                        r <= 512 (at temp > 0 also r <= 256 when Nmax > 32)
+ *                        and the device can hold one such CTA per SM,
+ *                        otherwise one GEMM and one frontier launch per wave
+ *                        (the default);
  *   DT_BUILD_WAVES       always one launch pair per wave;
  *   DT_BUILD_PERSISTENT  always the persistent launch: calls that do not fit
  *                        it return DT_EUNSUPPORTED with nothing enqueued.

@@ -11,13 +11,13 @@ only reach in miniature, and of the build on non-dyadic bf16 inputs.
 * TreeFlash (TreeFlash explainer, method sections 1-2): d = d_ff = 2560,
   V = 151936, gamma = 16, M = 4, budget 16, batch 16.  The GPU keeps the bf16
   activations the oracle's store hook models but sums in another order, so a
-  bf16 activation can round the other way (a logit moves by ~1e-4).  Requests
-  whose decision margins clear 1e-3 must give the oracle's tree exactly; at
-  this size about half of them have some decision closer than that (key gaps
-  among ~60 candidates), and for those the GPU tree is checked to be a valid
-  answer: each node among its parent's top M up to 1e-3, its key the oracle's
-  path key, and the tree the best-first top-budget set up to 1e-3.  Both
-  counts are printed; every request is checked one way or the other.
+  bf16 activation can round the other way (a logit moves by up to ~2e-3, see
+  TF_TOL).  Requests whose decision margins clear TF_TOL must give the
+  oracle's tree exactly; for the others (some decision closer than that: key
+  gaps among ~60 candidates) the GPU tree is checked to be a valid answer:
+  each node among its parent's top M up to TF_TOL, its key the oracle's path
+  key, and the tree the best-first top-budget set up to TF_TOL.  Both counts
+  are printed; every request is checked one way or the other.
 * Non-dyadic build (PCTree summary, DSpark paragraph): the Qwen3-4B-shaped
   round with plain bf16 Markov factors and block logits, so the tensor-core
   logits are no longer exact in fp32.  Seeds whose top-k, key-order and
@@ -144,7 +144,16 @@ def _tf_margin(W, x, b, M, tree, dist):
     return min(gaps)
 
 
-def _tf_valid(x, b, M, out, tree, sets, dist, tol=1e-3):
+# TreeFlash decisions ride on bf16 activations: one bf16 ulp of an element of
+# the residual stream h' (|h'| up to ~4, ulp 2^-6) times an LM-head weight
+# (~0.02) moves a logit by ~3e-4, and a few such rounding flips on either side
+# reach ~2e-3.  Decisions closer than TF_TOL are checked for validity rather
+# than compared; keys agree within TF_TOL (+ 1e-4 |key| over the depth), all
+# well inside the 2e-2 absolute tolerance for bf16 logits.
+TF_TOL = 5e-3
+
+
+def _tf_valid(x, b, M, out, tree, sets, dist, tol=TF_TOL):
     """Where a near-tie may flip a decision, check that the GPU tree of request
     b is one of the valid answers: structure consistent, each node among the
     top M of its parent's oracle distribution and of its depth's stage-1 set
@@ -175,7 +184,9 @@ def _tf_valid(x, b, M, out, tree, sets, dist, tol=1e-3):
         sd, lse = dist[(int(dep[i]), prev)]
         v = np.sort(sd)[::-1]
         assert sd[tok[i]] >= v[M - 1] - tol, (b, i)
-        assert abs(keys[i] - (kp + sd[tok[i]] - lse)) <= tol, (b, i)
+        # the key tolerance of the exact comparison: TF_TOL + 1e-4 |key|
+        ref = kp + sd[tok[i]] - lse
+        assert abs(keys[i] - ref) <= tol + 1e-4 * abs(ref), (b, i, float(keys[i]), ref)
     # best-first: nothing left out beats the tree's weakest node (up to tol)
     members = {(int(dep[i]), int(tok[i]), int(par[i])) for i in range(n)}
     parents = [(-1, root, 0, 0.0)] + [(i, int(tok[i]), int(dep[i]), float(keys[i]))
@@ -214,8 +225,8 @@ def test_treeflash_full_size():
         assert all(len(set(int(t) for t in s)) == M for s in sets)
         assert len(dist) <= M * gamma
         margin = _tf_margin(W, x, b, M, tree, dist)
-        if margin <= 1e-3:
-            # a decision within 1e-3: either answer is correct, check validity
+        if margin <= TF_TOL:
+            # a decision within TF_TOL: either answer is correct, check validity
             near.append((b, margin))
             _tf_valid(x, b, M, out, tree, sets, dist)
             continue
@@ -228,7 +239,9 @@ def test_treeflash_full_size():
         assert np.array_equal(g(out.depths), tree.depths), b
         assert np.array_equal(g(out.ranks), tree.ranks), b
         assert np.array_equal(g(out.anc).astype(np.uint64), tree.anc), b
-        assert np.allclose(g(out.keys), tree.keys64, atol=1e-3, rtol=0), b
+        # a key sums depth-many log-probabilities, each with its own bf16
+        # activation rounding: relative 1e-4 on top of TF_TOL
+        assert np.allclose(g(out.keys), tree.keys64, atol=TF_TOL, rtol=1e-4), b
     print(f"treeflash full size: {exact} of {batch} requests compared exactly, "
           f"{len(near)} checked for validity at near-ties {near}")
     assert exact + len(near) == batch
