@@ -112,6 +112,25 @@ def oracle_inputs(w, target):
                 attn=attention_inputs(w, w.Nmax + 1, 0), target=target.astype(np.float64))
 
 
+def time_cpu_round(w, target, budget_s=10.0):
+    """The oracle's greedy round restated in C++ (fp64, OpenMP on every host
+    core), on the same inputs as time_oracle: rounds/s, rounds, seconds."""
+    from gen import attention_inputs
+    from oracle import cpu_round
+    attn = attention_inputs(w, w.Nmax + 1, 0)
+    run = lambda: cpu_round.round_t0(w.L[0], w.A, w.Bt, w.root[0], w.k, w.Nmax, attn,
+                                     1.0 / math.sqrt(w.d), target)
+    run()  # compiles (first use on this host) and warms
+    n, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return n / el, n, el
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -539,6 +558,13 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_oracle and args.workload == WORKLOAD:
         v, nr, el = time_oracle(w, tgt[0], budget_s=20.0)
+        vc, nc, elc = time_cpu_round(w, tgt[0], budget_s=10.0)
+        from oracle import cpu_round
+        out["cpu_baseline_openmp"] = {
+            "value": round(vc, 3), "unit": UNIT, "cores": cpu_round.threads(),
+            "kind": "oracle restated in C++ (fp64, -O3 -march=native, OpenMP)",
+            "sample": f"{nc} full rounds of the same workload in {elc:.1f} s "
+                      "(build + verify + accept, request 0)"}
         out["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": blas_threads(),
                                "kind": "oracle",
                                "sample": f"{nr} full rounds of the same workload in {el:.1f} s "
