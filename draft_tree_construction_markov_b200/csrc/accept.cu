@@ -31,6 +31,24 @@ __device__ __forceinline__ float ld_logit(const void* base, int bf16, size_t i) 
   return bf16 ? bf16_to_f32(((const uint16_t*)base)[i]) : ((const float*)base)[i];
 }
 
+// Four consecutive logits from index i (a multiple of 4; the row is 16-byte
+// aligned in fp32 and 8-byte aligned in bf16).
+__device__ __forceinline__ void ld_logit4(const void* base, int bf16, size_t i, float (&v)[4]) {
+  if (bf16) {
+    const uint2 u = __ldg((const uint2*)((const uint16_t*)base + i));
+    v[0] = __uint_as_float(u.x << 16);
+    v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16);
+    v[3] = __uint_as_float(u.y & 0xffff0000u);
+  } else {
+    const float4 f = __ldg((const float4*)((const float*)base + i));
+    v[0] = f.x;
+    v[1] = f.y;
+    v[2] = f.z;
+    v[3] = f.w;
+  }
+}
+
 struct AccParts {
   float* pv;    // [rows_total][splits] argmax value or (T>0) max
   int32_t* pi;  // [rows_total][splits] argmax id
@@ -318,6 +336,7 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
   __shared__ float red[32];
   __shared__ int32_t redi[32];
   __shared__ int kids[64];
+  __shared__ int32_t s_removed[64];  // tokens of the rejected siblings, in order
   __shared__ int s_nk, s_acc;
   __shared__ float s_lse;
   __shared__ int32_t s_tok[64], s_par[64], s_rank[64];
@@ -336,7 +355,12 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
   }
   __syncthreads();
   const int V = w.V;
-  const int chunk = (V + C - 1) / C;
+  // Vector mode: rows of a multiple of 4 tokens on 16-byte boundaries, read
+  // and written four tokens per load; every slice starts on a multiple of 4.
+  const bool vec = (V & 3) == 0 && ((uintptr_t)w.t & 15) == 0 && ((uintptr_t)w.draft_q & 15) == 0 &&
+                   ((uintptr_t)w.rbuf & 15) == 0;
+  const int sh = vec ? 2 : 0;  // log2 of the tokens a thread reads at once
+  const int chunk = vec ? ((V + 4 * C - 1) / (4 * C)) * 4 : (V + C - 1) / C;
   const int v0 = min(V, rank * chunk), v1 = min(V, v0 + chunk);  // this CTA's slice
   const float temp = w.temp;
   float* rb[2] = {w.rbuf + (size_t)b * 2 * V, w.rbuf + (size_t)b * 2 * V + V};
@@ -382,12 +406,26 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
     int cur = 0;         // residual buffer holding p (unnormalised) when resid
     float zr = 1.f;      // normaliser of the residual
     float qn = 1.f;      // sum of q over the tokens not yet removed
-    int removed[16];
+    // The removed set is the first n_removed entries of s_removed (at most nk,
+    // and a node has fewer than Nmax <= 64 children).  A pass looks up the
+    // removed tokens that fall in this thread's groups of the slice (group g
+    // = (y - v0) >> sh belongs to thread g % kWalkThreads) only when it
+    // reaches the previous one, and meets them in ascending order as y
+    // advances.
     int n_removed = 0;
+    auto next_owned = [&](int after) {
+      int best = 0x7fffffff;
+      for (int i = 0; i < n_removed; ++i) {
+        const int t = s_removed[i];
+        if (t > after && t >= v0 && t < v1 && ((t - v0) >> sh) % kWalkThreads == tid)
+          best = min(best, t);
+      }
+      return best;
+    };
     for (int ci = 0; ci < nk; ++ci) {
       const int c = kids[ci];
       const int x = s_tok[c];
-      const float px = resid ? rb[cur][x] / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + x), temp) - lse_t);
+      const float px = resid ? __ldcg(rb[cur] + x) / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + x), temp) - lse_t);
       const float qx = q[x] / qn;
       const float u = philox_uniform(w.seed, w.offset, 1u, (uint32_t)b, (uint32_t)c, 0u, 0u);
       if (u < px / qx) {
@@ -396,20 +434,58 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
       }
       // residual pass over this CTA's slice: r'(y) = max(p(y) - q_j(y), 0),
       // q_j = q without the tokens removed before x, over the normaliser qn
-      removed[n_removed++] = x;
+      if (tid == 0) s_removed[n_removed] = x;
+      ++n_removed;
+      __syncthreads();
       float* dst = rb[cur ^ 1];
       float zsum = 0.f, qsum = 0.f;
-      for (int y = v0 + tid; y < v1; y += kWalkThreads) {
-        const float py =
-            resid ? rb[cur][y] / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + y), temp) - lse_t);
-        bool rm = false;
-        for (int i = 0; i < n_removed; ++i) rm |= (removed[i] == y);
-        const float qy = rm ? 0.f : q[y];
-        // q_j(y) uses the normaliser before this token was removed
-        const float rv = fmaxf(py - (rm && y != x ? 0.f : (y == x ? q[y] : qy)) / qn, 0.f);
-        dst[y] = rv;
+      int nxt = next_owned(-1);
+      // one token: p(y), then r'(y) = max(p(y) - q_j(y), 0) with q_j(y) = 0
+      // for tokens removed before x, over the normaliser qn
+      auto resid_one = [&](int y, float praw, float qv) {
+        const float py = resid ? praw / zr : expf(__fdiv_rn(praw, temp) - lse_t);
+        const bool rm = (y == nxt);
+        if (rm) nxt = next_owned(y);
+        const float rv = fmaxf(py - (rm && y != x ? 0.f : qv) / qn, 0.f);
         zsum += rv;
-        if (!rm) qsum += qy;
+        if (!rm) qsum += qv;
+        return rv;
+      };
+      if (vec) {
+        constexpr int kU = 2;  // groups of 4 tokens in flight per thread
+        const int g1 = v1 >> 2;
+        for (int g = (v0 >> 2) + tid; g < g1; g += kU * kWalkThreads) {
+          float pr[kU][4], qr[kU][4];
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int gg = g + u * kWalkThreads;
+            if (gg < g1) {
+              if (resid) {
+                const float4 f = __ldcg((const float4*)rb[cur] + gg);
+                pr[u][0] = f.x, pr[u][1] = f.y, pr[u][2] = f.z, pr[u][3] = f.w;
+              } else {
+                ld_logit4(w.t, w.tbf16, tbase + 4 * (size_t)gg, pr[u]);
+              }
+              const float4 f = __ldg((const float4*)q + gg);
+              qr[u][0] = f.x, qr[u][1] = f.y, qr[u][2] = f.z, qr[u][3] = f.w;
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int gg = g + u * kWalkThreads;
+            if (gg < g1) {
+              float4 o;
+              o.x = resid_one(4 * gg, pr[u][0], qr[u][0]);
+              o.y = resid_one(4 * gg + 1, pr[u][1], qr[u][1]);
+              o.z = resid_one(4 * gg + 2, pr[u][2], qr[u][2]);
+              o.w = resid_one(4 * gg + 3, pr[u][3], qr[u][3]);
+              __stcg((float4*)dst + gg, o);
+            }
+          }
+        }
+      } else {
+        for (int y = v0 + tid; y < v1; y += kWalkThreads)
+          dst[y] = resid_one(y, resid ? rb[cur][y] : ld_logit(w.t, w.tbf16, tbase + y), q[y]);
       }
       const WalkPart tot = cluster_sum2(cl, zsum, qsum, xs, slot, red, &bcast);
       slot ^= 1;
@@ -432,16 +508,40 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
     // bonus: exponential race argmax_y p(y) / E_y over every slice
     float best = -INFINITY;
     int32_t bid = 0x7fffffff;
-    for (int y = v0 + tid; y < v1; y += kWalkThreads) {
-      const float py =
-          resid ? rb[cur][y] / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + y), temp) - lse_t);
-      const float u = philox_uniform(w.seed, w.offset, 2u, (uint32_t)b, (uint32_t)(node + 1), 0u,
-                                     (uint32_t)y);
+    // one token: its race score p(y) / E_y, E_y = -log U_y
+    auto race_one = [&](int y, float praw, float u) {
+      const float py = resid ? praw / zr : expf(__fdiv_rn(praw, temp) - lse_t);
       const float sc = py / (-logf(u));
       if (sc > best) {
         best = sc;
         bid = y;
       }
+    };
+    if (vec) {
+      // the four tokens of a group share one Philox block (word y & 3)
+      const int g1 = v1 >> 2;
+      const uint32_t key0 = (uint32_t)w.seed, key1 = (uint32_t)(w.seed >> 32);
+      for (int g = (v0 >> 2) + tid; g < g1; g += kWalkThreads) {
+        float pr[4];
+        if (resid) {
+          const float4 f = __ldcg((const float4*)rb[cur] + g);
+          pr[0] = f.x, pr[1] = f.y, pr[2] = f.z, pr[3] = f.w;
+        } else {
+          ld_logit4(w.t, w.tbf16, tbase + 4 * (size_t)g, pr);
+        }
+        const U4 o = philox10(U4{(uint32_t)g | ((uint32_t)b << 18) | (2u << 28),
+                                 (uint32_t)(node + 1), 0u, w.offset},
+                              key0, key1);
+        race_one(4 * g, pr[0], u23(o.x));
+        race_one(4 * g + 1, pr[1], u23(o.y));
+        race_one(4 * g + 2, pr[2], u23(o.z));
+        race_one(4 * g + 3, pr[3], u23(o.w));
+      }
+    } else {
+      for (int y = v0 + tid; y < v1; y += kWalkThreads)
+        race_one(y, resid ? rb[cur][y] : ld_logit(w.t, w.tbf16, tbase + y),
+                 philox_uniform(w.seed, w.offset, 2u, (uint32_t)b, (uint32_t)(node + 1), 0u,
+                                (uint32_t)y));
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) {

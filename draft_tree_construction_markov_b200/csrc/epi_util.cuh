@@ -92,6 +92,27 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Whether the Gumbel key s + G, G = -log(-log U), U = ((word >> 9) + 0.5) 2^-23,
+// can exceed thr, decided without the two accurate logarithms of the key:
+// s + G > thr  <=>  w = -log U < exp(s - thr).
+//  * w is bounded below by v = 1 - U (exact in fp32) when v < 2^-7, since
+//    -log(1 - v) >= v, and otherwise by 0.999 (-__logf(U)): __logf's error
+//    (below 2^-21 absolute near 1, 2^-21 relative elsewhere) is far below
+//    0.1 % of w >= 2^-7.
+//  * exp(s - thr) is bounded above by 2^((s - thr) log2(e) + log2(1.001))
+//    with ex2.approx (relative error near 2^-22).
+// The two factors leave about 1e-3 of room on G, far more than the fp32
+// rounding of the key, so every token whose computed key beats thr passes,
+// and the caller computes the exact key for those only.  thr = -inf passes
+// every finite s; s = -inf never passes.
+__device__ __forceinline__ bool gumbel_may_beat(float s, float thr, uint32_t word) {
+  const uint32_t m = word >> 9;
+  const float v = ((float)(0x7fffffu - m) + 0.5f) * 1.1920928955078125e-07f;  // 1 - U
+  const float wlo =
+      v < 0.0078125f ? v : -0.999f * __logf(((float)m + 0.5f) * 1.1920928955078125e-07f);
+  return wlo < ex2_approx((s - thr) * kLog2e + 0.0014419741f);
+}
+
 __device__ __forceinline__ float load_bias1(const void* L, int bf16, int64_t off) {
   return bf16 ? bf16_to_f32(__ldg((const uint16_t*)L + off)) : __ldg((const float*)L + off);
 }

@@ -713,23 +713,26 @@ __global__ void __launch_bounds__(GemmShape<NG>::kThreads, 1)
             }
           }
           if constexpr (STOCH) {
-            // Gumbel keys; four consecutive tokens share one Philox counter
+            // Gumbel keys; four consecutive tokens share one Philox counter.
+            // The block's eight draws are independent and issued together;
+            // the exact key is computed only where it may beat the bar.
             if (mt + kGumbelMax > gthr[j]) {
+              uint32_t wds[32];
   #pragma unroll
               for (int gi = 0; gi < 8; ++gi) {
-                const float smax =
-                    fmaxf(fmaxf(s[4 * gi], s[4 * gi + 1]), fmaxf(s[4 * gi + 2], s[4 * gi + 3]));
-                if (!(smax + kGumbelMax > gthr[j])) continue;
                 const uint32_t x4 = (uint32_t)(a.v_base + xq + 4 * gi);
                 const U4 o = philox10(
                     U4{(x4 >> 2) | ((uint32_t)mc[j].b << 18), mc[j].c1, mc[j].c2, a.offset},
                     (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
-                const uint32_t wds[4] = {o.x, o.y, o.z, o.w};
+                wds[4 * gi] = o.x;
+                wds[4 * gi + 1] = o.y;
+                wds[4 * gi + 2] = o.z;
+                wds[4 * gi + 3] = o.w;
+              }
   #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                  const int i = 4 * gi + jj;
-                  if (i >= nv) continue;
-                  const float gk = s[i] + (-logf(-logf(u23(wds[jj]))));
+              for (int i = 0; i < 32; ++i) {
+                if (i < nv && gumbel_may_beat(s[i], gthr[j], wds[i])) {
+                  const float gk = s[i] + (-logf(-logf(u23(wds[i]))));
                   if (gk > gthr[j]) {
                     topk_insert<KMAX>(L2[j], I2[j], gk, a.v_base + xq + i);
                     gthr[j] = kth<KMAX>(L2[j], k);

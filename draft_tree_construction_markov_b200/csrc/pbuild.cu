@@ -20,18 +20,23 @@
 // the 148 per-CTA partials of every node on a single CTA.  Here:
 //  * one CTA per SM owns a contiguous vocabulary range of Bm for the whole
 //    build.  Its block-logit rows (every request and depth) are loaded once.
-//  * a producer thread streams the range through a TMA stage ring that runs
-//    ahead across waves, so the next wave's first tiles are in flight while
-//    the current wave is merged and selected.  The loads carry an L2
+//  * a producer thread streams the range through a TMA stage ring.  Each
+//    wave's pass over the range is released as soon as the previous wave's
+//    merged rows are read, so its first tiles are in flight while the
+//    selection that decides its nodes still runs.  The loads carry an L2
 //    evict-last hint: waves 2.. re-read the same 78 MB.
 //  * after its epilogue every CTA writes one partial per node and meets the
-//    others at a grid barrier (bounded wait).  Then EVERY CTA merges every
-//    node's partials and runs the selection itself: all read the same bytes
-//    and take the same decisions in the same order, so the next wave's nodes
-//    need no second barrier.  CTA 0 writes the tree.
+//    others at a grid barrier (bounded wait).  The merge of a node row's
+//    per-CTA partials is then spread over the grid: row e is merged by CTA
+//    e % ncta alone (148 CTAs reading the same lines at once would queue on
+//    the same L2 slices), which writes the row's log-sum-exp and k best
+//    entries to a merged-row buffer.  After a second grid barrier EVERY CTA
+//    reads the merged rows and runs the selection itself: all read the same
+//    bytes and take the same decisions in the same order, so the next wave's
+//    nodes need no further exchange.  CTA 0 writes the tree.
 //  * partial buffers alternate by wave parity: a CTA can only write wave
-//    w + 2's partials after every CTA has passed barrier w + 1, i.e. has
-//    finished merging wave w.
+//    w + 2's partials after every CTA has passed the barriers of wave w + 1,
+//    i.e. has finished merging wave w.
 #include "build.cuh"
 #include "epi_util.cuh"
 #include "merge.cuh"
@@ -890,23 +895,26 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
                 ssum += st * ex2_approx((mt - m) * kLog2e);
               }
               if constexpr (STOCH) {
-                // Gumbel keys; four consecutive tokens share one Philox counter
+                // Gumbel keys; four consecutive tokens share one Philox counter.
+                // The block's eight draws are independent and issued together;
+                // the exact key is computed only where it may beat the bar.
                 if (mt + kGumbelMax > gthr) {
+                  uint32_t wds[32];
 #pragma unroll
                   for (int gi = 0; gi < 8; ++gi) {
-                    const float smax = fmaxf(fmaxf(sv[4 * gi], sv[4 * gi + 1]),
-                                             fmaxf(sv[4 * gi + 2], sv[4 * gi + 3]));
-                    if (!(smax + kGumbelMax > gthr)) continue;
                     const uint32_t x4 = (uint32_t)(xq + 4 * gi);
                     const U4 o =
                         philox10(U4{(x4 >> 2) | ((uint32_t)mc.b << 18), mc.c1, mc.c2, a.offset},
                                  (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
-                    const uint32_t wds[4] = {o.x, o.y, o.z, o.w};
+                    wds[4 * gi] = o.x;
+                    wds[4 * gi + 1] = o.y;
+                    wds[4 * gi + 2] = o.z;
+                    wds[4 * gi + 3] = o.w;
+                  }
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                      const int i = 4 * gi + jj;
-                      if (i >= nv) continue;
-                      const float gk = sv[i] + (-logf(-logf(u23(wds[jj]))));
+                  for (int i = 0; i < 32; ++i) {
+                    if (i < nv && gumbel_may_beat(sv[i], gthr, wds[i])) {
+                      const float gk = sv[i] + (-logf(-logf(u23(wds[i]))));
                       if (gk > gthr) {
                         topk_insert<KMAX>(L2, I2, gk, xq + i);
                         gthr = kth<KMAX>(L2, k);

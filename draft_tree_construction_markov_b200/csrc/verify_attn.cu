@@ -6,20 +6,15 @@
 // root's tree row, and tree row j+1 iff node j is node i-1 or one of its
 // ancestors (bit j of anc[b][i-1]).
 //
-// bf16 path: split-KV ("flash-decoding") over 64-column chunks.  A CTA owns one
-// (request, KV head, column split, row block); its query rows are the G = Hq/Hkv
-// heads sharing the KV head times the tree rows, so every K/V chunk read from
-// HBM serves all of them.  Q.K^T and P.V run on warp-level bf16 MMAs with fp32
-// accumulation and an online softmax; the ancestor bitmask is applied only to
-// the tree columns.  A combine kernel merges the splits.  fp32 inputs use a
+// bf16 inputs: the tensor-core kernel of attn_tc.cu computes split-KV
+// partials (128 key columns per split; a CTA's rows are the query heads that
+// share one KV head times the tree rows, so every K/V tile read serves all of
+// them), and the combine kernel below merges the splits.  fp32 inputs use a
 // plain per-(row, head) kernel.
-#include <algorithm>
-
 #include "attn_tc.cuh"
 
 namespace dt {
 
-constexpr int kChunk = 64;
 constexpr float kAttnL2e = 1.4426950408889634f;
 
 struct AttnArgs {
@@ -47,244 +42,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-// 16-byte global -> shared copy that does not block the thread; zero-fills
-// the destination when `pred` is false.
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool pred) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(pred ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // Is tree column j (0 = root, j' + 1 = node j') visible from tree row i?
 __device__ __forceinline__ bool tree_visible(int i, int j, uint64_t anc_row) {
   return j == 0 || (i >= 1 && ((anc_row >> (j - 1)) & 1ull));
 }
 
-template <int D>
-__global__ void __launch_bounds__(512) attn_bf16_kernel(AttnArgs a) {
-  constexpr int LD = D + 8;  // padded row (bf16 elements) against bank conflicts
-  extern __shared__ __align__(16) uint8_t asmem[];
-  uint16_t* sQ = (uint16_t*)asmem;                 // [rows_per_cta][LD]
-  uint16_t* sKV = sQ + (size_t)a.rows_per_cta * LD; // 2 x ([kChunk][LD] K, [kChunk][LD] V)
-  const int split = blockIdx.x, kvh = blockIdx.y;
-  const int b = blockIdx.z / a.n_rblocks, rb = blockIdx.z % a.n_rblocks;
-  const int n = min(max(a.n_nodes[b], 0), a.Nmax);
-  const int P = min(max(a.plen[b], 0), a.max_prefix);
-  if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && rb == 0 &&
-      (a.n_nodes[b] != n || a.plen[b] != P))
-    set_status(a.status, DT_EDEVICE);
-  const int R = a.G * (n + 1);
-  const int row0 = rb * a.rows_per_cta;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nthreads = blockDim.x;
-  const int C = P + n + 1;
-  const int c0 = split * a.cols_per_split, c1 = min(C, c0 + a.cols_per_split);
-  const size_t pbase = (((size_t)split * a.batch + b) * a.Hkv + kvh) * (size_t)(a.n_rblocks * a.rpad) +
-                       row0;
-  if (row0 >= R) return;
-  // ---- Q rows of this block: rho = i * G + hh  ->  q[b][i][kvh*G + hh]
-  const uint16_t* q = (const uint16_t*)a.q;
-  for (int idx = tid; idx < a.rows_per_cta * (D / 8); idx += nthreads) {
-    const int rr = idx / (D / 8), cc = idx % (D / 8);
-    const int rho = row0 + rr;
-    const bool ok = rho < R;
-    const int i = ok ? rho / a.G : 0, hh = ok ? rho % a.G : 0;
-    cp_async16(sQ + (size_t)rr * LD + cc * 8,
-               q + (((size_t)b * (a.Nmax + 1) + i) * a.Hq + kvh * a.G + hh) * D + cc * 8, ok);
-  }
-  // per-lane rows (g and g + 8 of the warp's 16-row tile)
-  const int g = lane >> 2, t4 = lane & 3;
-  const int rloc0 = warp * 16 + g, rloc1 = rloc0 + 8;
-  const int rho0 = row0 + rloc0, rho1 = row0 + rloc1;
-  const int i0 = rho0 / a.G, i1 = rho1 / a.G;
-  const uint64_t anc0 = (rho0 < R && i0 >= 1) ? a.anc[(size_t)b * a.Nmax + i0 - 1] : 0ull;
-  const uint64_t anc1 = (rho1 < R && i1 >= 1) ? a.anc[(size_t)b * a.Nmax + i1 - 1] : 0ull;
-  const bool warp_active = warp * 16 < a.rows_per_cta;
-
-  float o[D / 8][4];
-#pragma unroll
-  for (int nt = 0; nt < D / 8; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  const float sl2 = a.scale * kAttnL2e;
-  const uint16_t* kp = (const uint16_t*)a.kp;
-  const uint16_t* vp = (const uint16_t*)a.vp;
-  const uint16_t* ktr = (const uint16_t*)a.kt;
-  const uint16_t* vtr = (const uint16_t*)a.vt;
-  const int64_t ps = a.pstart[b];
-
-  // K/V chunk loader: buffer `buf` <- columns [cb, cb + kChunk)
-  auto load_chunk = [&](int cb, int buf) {
-    uint16_t* dK = sKV + (size_t)buf * 2 * kChunk * LD;
-    uint16_t* dV = dK + kChunk * LD;
-    for (int idx = tid; idx < kChunk * (D / 8); idx += nthreads) {
-      const int rr = idx / (D / 8), cc = idx % (D / 8);
-      const int c = cb + rr;
-      const bool ok = c < c1;
-      size_t off;
-      const uint16_t *ks, *vs;
-      if (!ok) {  // zero-filled; the source is any valid address
-        off = 0;
-        ks = ktr;
-        vs = vtr;
-      } else if (c < P) {
-        off = ((size_t)(ps + c) * a.Hkv + kvh) * D + cc * 8;
-        ks = kp;
-        vs = vp;
-      } else {
-        off = (((size_t)b * (a.Nmax + 1) + (c - P)) * a.Hkv + kvh) * D + cc * 8;
-        ks = ktr;
-        vs = vtr;
-      }
-      cp_async16(dK + (size_t)rr * LD + cc * 8, ks + off, ok);
-      cp_async16(dV + (size_t)rr * LD + cc * 8, vs + off, ok);
-    }
-  };
-  if (c0 < c1) load_chunk(c0, 0);
-  cp_async_commit();  // group: Q + first chunk
-  int buf = 0;
-  for (int cb = c0; cb < c1; cb += kChunk, buf ^= 1) {
-    if (cb + kChunk < c1) load_chunk(cb + kChunk, buf ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();  // everything but the chunk just issued has landed
-    __syncthreads();
-    const uint16_t* sK = sKV + (size_t)buf * 2 * kChunk * LD;
-    const uint16_t* sV = sK + kChunk * LD;
-    if (warp_active) {
-    // S = Q K^T for 16 rows x 64 columns
-    float s[kChunk / 8][4];
-#pragma unroll
-    for (int nt = 0; nt < kChunk / 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t af[4];
-      ldsm_x4(af, smem_u32(sQ + (size_t)(warp * 16 + (lane & 15)) * LD + kk * 16 + (lane >> 4) * 8));
-#pragma unroll
-      for (int nt = 0; nt < kChunk / 8; nt += 2) {
-        uint32_t bf[4];
-        const int mi = lane >> 3, rr = lane & 7;
-        ldsm_x4(bf, smem_u32(sK + (size_t)(8 * (nt + (mi >> 1)) + rr) * LD + kk * 16 + (mi & 1) * 8));
-        mma_bf16_16816(s[nt], af, bf[0], bf[1]);
-        mma_bf16_16816(s[nt + 1], af, bf[2], bf[3]);
-      }
-    }
-    // mask + online softmax (rows rho0, rho1)
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < kChunk / 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = cb + nt * 8 + 2 * t4 + (e & 1);
-        const bool r1 = e >= 2;
-        const int rho = r1 ? rho1 : rho0;
-        bool ok = c < c1 && rho < R;
-        if (ok && c >= P) ok = tree_visible(r1 ? i1 : i0, c - P, r1 ? anc1 : anc0);
-        const float v = ok ? s[nt][e] * sl2 : -INFINITY;
-        s[nt][e] = v;
-        if (r1)
-          mx1 = fmaxf(mx1, v);
-        else
-          mx0 = fmaxf(mx0, v);
-      }
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float al0 = (mn0 == -INFINITY) ? 1.f : exp2f(m0 - mn0);
-    const float al1 = (mn1 == -INFINITY) ? 1.f : exp2f(m1 - mn1);
-    float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < kChunk / 8; ++nt) {
-      s[nt][0] = (mn0 == -INFINITY) ? 0.f : exp2f(s[nt][0] - mn0);
-      s[nt][1] = (mn0 == -INFINITY) ? 0.f : exp2f(s[nt][1] - mn0);
-      s[nt][2] = (mn1 == -INFINITY) ? 0.f : exp2f(s[nt][2] - mn1);
-      s[nt][3] = (mn1 == -INFINITY) ? 0.f : exp2f(s[nt][3] - mn1);
-      rs0 += s[nt][0] + s[nt][1];
-      rs1 += s[nt][2] + s[nt][3];
-    }
-    l0 = l0 * al0 + rs0;  // per-lane partial row sums; reduced over the quad at the end
-    l1 = l1 * al1 + rs1;
-    m0 = mn0;
-    m1 = mn1;
-#pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt) {
-      o[nt][0] *= al0;
-      o[nt][1] *= al0;
-      o[nt][2] *= al1;
-      o[nt][3] *= al1;
-    }
-    // O += P V
-#pragma unroll
-    for (int kk = 0; kk < kChunk / 16; ++kk) {
-      uint32_t af[4];
-      af[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-      af[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-      af[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      af[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-#pragma unroll
-      for (int nt = 0; nt < D / 8; nt += 2) {
-        uint32_t bf[4];
-        const int mi = lane >> 3, rr = lane & 7;
-        ldsm_x4_t(bf, smem_u32(sV + (size_t)(kk * 16 + (mi & 1) * 8 + rr) * LD + 8 * (nt + (mi >> 1))));
-        mma_bf16_16816(o[nt], af, bf[0], bf[1]);
-        mma_bf16_16816(o[nt + 1], af, bf[2], bf[3]);
-      }
-    }
-    }  // warp_active
-    __syncthreads();  // buffer `buf` is refilled by the next iteration's loads
-  }
-  cp_async_wait<0>();
-  if (!warp_active) return;
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  if (rloc0 < a.rows_per_cta && rho0 < R) {
-    float* po = a.part_o + (pbase + rloc0) * D;
-#pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt)
-      *(float2*)(po + nt * 8 + 2 * t4) = make_float2(o[nt][0], o[nt][1]);
-    if (t4 == 0) a.part_ml[pbase + rloc0] = make_float2(m0, l0);
-  }
-  if (rloc1 < a.rows_per_cta && rho1 < R) {
-    float* po = a.part_o + (pbase + rloc1) * D;
-#pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt)
-      *(float2*)(po + nt * 8 + 2 * t4) = make_float2(o[nt][2], o[nt][3]);
-    if (t4 == 0) a.part_ml[pbase + rloc1] = make_float2(m1, l1);
-  }
-}
 
 constexpr int kMaxSplits = 512;
 constexpr int kCombineWarps = 4;
@@ -435,7 +198,7 @@ __global__ void attn_f32_kernel(AttnArgs a, int max_cols) {
 }
 
 struct AttnPlan {
-  int splits, cols_per_split, rows_per_cta, n_rblocks, rpad, warps;
+  int splits, cols_per_split, rows_per_cta, n_rblocks, rpad;
   size_t part_o_bytes, part_ml_bytes;
 };
 
@@ -446,33 +209,9 @@ static AttnPlan attn_tc_plan(int batch, int Nmax, int Hq, int Hkv, int d, int ma
   const int G = Hq / Hkv;
   p.n_rblocks = 1;
   p.rows_per_cta = p.rpad = G * (Nmax + 1);
-  p.warps = 4;
   p.cols_per_split = 128;
   p.splits = (max_prefix + Nmax + 1 + 127) / 128;
   const size_t rows = (size_t)p.splits * batch * Hkv * p.rpad;
-  p.part_o_bytes = rows * d * 4;
-  p.part_ml_bytes = rows * 8;
-  return p;
-}
-
-static AttnPlan attn_plan(int batch, int Nmax, int Hq, int Hkv, int d, int max_prefix) {
-  AttnPlan p;
-  const int G = Hq / Hkv;
-  const int Rmax = G * (Nmax + 1);
-  p.n_rblocks = (Rmax + 255) / 256;
-  const int per = (Rmax + p.n_rblocks - 1) / p.n_rblocks;
-  p.warps = (per + 15) / 16;
-  p.rows_per_cta = p.warps * 16;
-  p.rpad = p.rows_per_cta;
-  const int Cmax = max_prefix + Nmax + 1;
-  const int chunks = (Cmax + kChunk - 1) / kChunk;
-  const int base_ctas = batch * Hkv * p.n_rblocks;
-  int want = (148 + base_ctas - 1) / base_ctas;
-  want = std::max(1, std::min(want, chunks));
-  const int chunks_per = (chunks + want - 1) / want;
-  p.cols_per_split = chunks_per * kChunk;
-  p.splits = (chunks + chunks_per - 1) / chunks_per;  // at most 2 * 148 <= kMaxSplits
-  const size_t rows = (size_t)p.splits * batch * Hkv * p.n_rblocks * p.rpad;
   p.part_o_bytes = rows * d * 4;
   p.part_ml_bytes = rows * 8;
   return p;
@@ -488,11 +227,8 @@ size_t dt_tree_verify_attn_workspace_bytes(int batch, int Nmax, int Hq, int Hkv,
                                            int max_prefix) {
   if (batch <= 0 || Nmax <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || d <= 0 || max_prefix < 0)
     return 0;
-  AttnPlan p = attn_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
-  AttnPlan t = attn_tc_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
-  const size_t ml = std::max(p.part_ml_bytes, t.part_ml_bytes);
-  const size_t o = std::max(p.part_o_bytes, t.part_o_bytes);
-  return kWsHeader + ((ml + 255) & ~(size_t)255) + o + 256;
+  const AttnPlan t = attn_tc_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
+  return kWsHeader + ((t.part_ml_bytes + 255) & ~(size_t)255) + t.part_o_bytes + 256;
 }
 
 dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const void* d_v_prefix,
@@ -513,9 +249,7 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const voi
   if (!ws || ws_bytes < need) return DT_EWORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   // bf16: the tensor-core kernel; fp32 inputs: the plain per-(row, head) kernel
-  const bool tc = dt == DT_BF16;
-  AttnPlan p = tc ? attn_tc_plan(batch, Nmax, Hq, Hkv, d, max_prefix)
-                  : attn_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
+  const AttnPlan p = attn_tc_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
   AttnArgs a;
   a.q = d_q;
   a.kp = d_k_prefix;
@@ -541,12 +275,8 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const voi
   a.rpad = p.rpad;
   uint8_t* w = (uint8_t*)ws;
   a.status = (int32_t*)w;
-  {
-    AttnPlan p0 = attn_plan(batch, Nmax, Hq, Hkv, d, max_prefix);
-    const size_t ml = std::max(p0.part_ml_bytes, p.part_ml_bytes);
-    a.part_ml = (float2*)(w + kWsHeader);
-    a.part_o = (float*)(w + kWsHeader + ((ml + 255) & ~(size_t)255));
-  }
+  a.part_ml = (float2*)(w + kWsHeader);
+  a.part_o = (float*)(w + kWsHeader + ((p.part_ml_bytes + 255) & ~(size_t)255));
   a.out = d_out;
   a.out_bf16 = dt == DT_BF16;
   if (cudaMemsetAsync(a.status, 0, 4, s) != cudaSuccess) return DT_ECUDA;
@@ -592,13 +322,9 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix, const voi
   ProfileScope ps(DT_K_ATTN_COMBINE, s);
   const int items = batch * (Nmax + 1) * Hq;
   const dim3 cgrid((items + kCombineWarps - 1) / kCombineWarps);
-  if (tc) {
-    // launched while the attention kernel runs; it waits for its partials
-    if (launch_pdl(attn_combine_kernel, cgrid, dim3(32 * kCombineWarps), 0, s, a) != cudaSuccess)
-      return DT_ECUDA;
-  } else {
-    attn_combine_kernel<<<cgrid, 32 * kCombineWarps, 0, s>>>(a);
-  }
+  // launched while the attention kernel runs; it waits for its partials
+  if (launch_pdl(attn_combine_kernel, cgrid, dim3(32 * kCombineWarps), 0, s, a) != cudaSuccess)
+    return DT_ECUDA;
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ECUDA;
 }
 

@@ -34,6 +34,7 @@ ACCEPT_CASES = [
     ("tiny", {}, 1.0),
     ("tiny", dict(V=1000, r=32, Bk=5, k=3, N=20), 0.7),
     ("tiny", dict(V=1000, r=32, Bk=5, k=3, N=20, batch=3), 2.0),
+    ("tiny", dict(V=777, r=48, Bk=6, k=5, N=40), 1.3),  # V % 4 != 0: the walk's scalar path
     ("qwen3_4b", {}, 0.0),
     ("qwen3_8b", {}, 0.6),
 ]
@@ -190,3 +191,66 @@ def test_emitted_tokens_follow_target_chi_square(temp):
     assert by_first[y1].sum() > 10000
     p1 = accept.softmax(tab[1, y1].astype(np.float64) / temp)
     assert chi(by_first[y1], p1) > 0.01
+
+
+def test_stochastic_walk_wide_node():
+    """A node with 40 children, more rejected siblings than any build emits.
+
+    The walk keeps the whole removed-sibling set (up to Nmax - 1 tokens) and
+    its residuals stay those of the oracle: requests 0-2 reject all 40
+    children, requests 3-5 reject 30 and accept the 31st.
+    """
+    B, V, Nmax, nk, Bk, temp = 6, 20000, 48, 40, 2, 1.0
+    rng = np.random.default_rng(41)
+    tokens = np.stack([rng.choice(V, nk, replace=False) for _ in range(B)]).astype(np.int32)
+    t = np.zeros((B, Nmax + 1, V), np.float32)
+    q = np.zeros((B, Nmax + 1, V), np.float32)
+    for b in range(B):
+        t[b, : nk + 1] = rng.standard_normal((nk + 1, V))
+        t[b, 0, tokens[b]] = -30.0
+        if b >= 3:
+            t[b, 0, tokens[b, 30]] = 12.0
+        q0 = np.full(V, 0.7 / (V - nk))
+        q0[tokens[b]] = 0.3 / nk
+        q[b, 0] = (q0 / q0.sum()).astype(np.float32)
+    tree = dt.Tree.empty(B, Nmax, V, stochastic=True)
+    pad = np.zeros((B, Nmax), np.int32)
+    tok = pad.copy()
+    tok[:, :nk] = tokens
+    par = np.full((B, Nmax), -1, np.int32)
+    dep = pad.copy()
+    dep[:, :nk] = 1
+    rnk = pad.copy()
+    rnk[:, :nk] = np.arange(nk)
+    tree.tokens.copy_(torch.from_numpy(tok))
+    tree.parents.copy_(torch.from_numpy(par))
+    tree.depths.copy_(torch.from_numpy(dep))
+    tree.ranks.copy_(torch.from_numpy(rnk))
+    tree.n_nodes.fill_(nk)
+    tree.draft_q.copy_(torch.from_numpy(q))
+    acc = torch.empty(B, Bk, dtype=torch.int32, device="cuda")
+    nacc = torch.empty(B, dtype=torch.int32, device="cuda")
+    bonus = torch.empty(B, dtype=torch.int32, device="cuda")
+    ws = dt.workspace(dt.accept_workspace_bytes(B, Nmax, V))
+    dt.tree_accept(dev(t), tree, Bk, temp, acc, nacc, bonus, ws, philox_seed=5, philox_offset=2)
+    assert dt.read_status(ws) == 0
+    acc, nacc, bonus = acc.cpu().numpy(), nacc.cpu().numpy(), bonus.cpu().numpy()
+    compared = 0
+    for b in range(B):
+        o = markov_tree.Tree(
+            tokens=tokens[b], parents=np.full(nk, -1, np.int32), depths=np.ones(nk, np.int32),
+            ranks=np.arange(nk, dtype=np.int32), keys=np.zeros(nk, np.float32),
+            keys64=np.zeros(nk), anc=(np.uint64(1) << np.arange(nk, dtype=np.uint64)),
+            expansions={}, margins=[])
+        margins = []
+        path, bon = accept.stochastic_walk(o, t[b, : nk + 1].astype(np.float64), temp, seed=5,
+                                           offset=2, request=b, q_rows={0: q[b, 0]},
+                                           margins=margins)
+        assert path == ([] if b < 3 else [30]), (b, path)
+        if min(m[1] for m in margins) < 1e-4:
+            continue  # a coin or race within fp32 rounding of its threshold
+        compared += 1
+        assert nacc[b] == len(path) and acc[b, : nacc[b]].tolist() == path, b
+        assert np.all(acc[b, nacc[b]:] == -1)
+        assert bonus[b] == bon, b
+    assert compared >= 4
