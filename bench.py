@@ -259,7 +259,7 @@ def peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def build_roofline(kern, *, V, r, B, Bk, inner, lbytes):
+def build_roofline(kern, *, V, r, B, Bk, inner, lbytes, waves=None):
     """Roofline object of the tree build, the round's dominant kernel.
 
     The algorithmic bytes are those of the whole build: the Markov factor Bm
@@ -269,6 +269,10 @@ def build_roofline(kern, *, V, r, B, Bk, inner, lbytes):
     few KB.  With the persistent build one launch is the whole build; with one
     launch pair per wave the GEMM launches of a round (Bk of them) together
     are, and each is charged Bm once, as if nothing stayed in L2 between them.
+
+    For the persistent build `stream` also states what the SMs move: every
+    one of the `waves` waves streams all of Bm, the first from HBM and the
+    others mostly from L2; that rate has no HBM denominator.
     """
     pk, pk_kind = peaks()
     flops = 2.0 * inner * V * r
@@ -300,6 +304,11 @@ def build_roofline(kern, *, V, r, B, Bk, inner, lbytes):
                  "algorithmic_bytes_per_launch": int(nbytes),
                  "algorithmic_flops_per_launch": int(flops),
                  "expanded_nodes_per_build": int(inner),
+                 **({"stream": {"waves": int(waves),
+                                "bytes_per_launch": int(waves * V * r * 2),
+                                "achieved_gbs": round(waves * V * r * 2 / (us * 1e-6) / 1e9, 1),
+                                "source": "Bm from HBM in the first wave, from L2 after"}}
+                    if "pbuild" in kern and waves else {}),
                  "traffic": traffic_from_profile(os.path.join(
                      ROOT, "draft_tree_construction_markov_b200", "csrc", src)),
                  "avg_launch_us": round(us, 3)})
@@ -394,11 +403,14 @@ def run_ours(args):
     tgt = np.zeros((B, N + 1, V), np.float32)
     n_nodes = tree.n_nodes.cpu().numpy()
     inner = 0
+    waves = 1
     for b in range(B):
         n = int(n_nodes[b])
         depths = tree.depths[b, :n].cpu().numpy()
         tokens = tree.tokens[b, :n].cpu().numpy()
         inner += 1 + int((depths < Bk).sum())
+        # wave w expands the nodes of depth w (the root in wave 0)
+        waves = max(waves, 1 + int(depths[depths < Bk].max(initial=0)))
         tgt[b, : n + 1] = target_rows(w, b, np.concatenate([[0], depths]),
                                       np.concatenate([w.root[b:b + 1], tokens]))
     for c in copies:
@@ -480,7 +492,7 @@ def run_ours(args):
     kern = {nm: {"launches_per_step": len(v) / kprof, "avg_us": 1e3 * statistics.mean(v),
                  "us_per_step": 1e3 * sum(v) / kprof} for nm, v in per_kind.items()}
 
-    roof = build_roofline(kern, V=V, r=r, B=B, Bk=Bk, inner=inner,
+    roof = build_roofline(kern, V=V, r=r, B=B, Bk=Bk, inner=inner, waves=waves,
                           lbytes=2 if w.logit_dtype == "bf16" else 4)
 
     # ---- end to end through the public API: pinned host inputs, copies timed

@@ -273,23 +273,6 @@ __global__ void __launch_bounds__(kPreThreads)
   }
 }
 
-template <int NT>
-__device__ __forceinline__ float block_sum(float v, float* red) {
-  v = warp_sum(v);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float r = 0.f;
-  if (warp == 0) {
-    r = lane < NT / 32 ? red[lane] : 0.f;
-    r = warp_sum(r);
-    if (lane == 0) red[0] = r;
-  }
-  __syncthreads();
-  return red[0];
-}
-
 // Stochastic walk, one thread-block cluster per request.  The C CTAs of the
 // cluster own consecutive slices of the vocabulary; a residual pass or the
 // bonus race runs over all slices at once, and its sums (or arg-max) are
@@ -303,18 +286,26 @@ struct __align__(8) WalkPart {
 };
 
 // Totals of (a, b) over the cluster, identical in every thread of every CTA:
-// block sums, then the CTAs' values combined by one fixed shuffle tree.
-// `slot` alternates between consecutive calls, so a slot is rewritten only
-// after a later cluster barrier has ordered every peer's read of it.
+// warp sums, the CTA's sum over its warps (warp 0), then the CTAs' values
+// combined by one fixed shuffle tree.  `slot` alternates between consecutive
+// calls, so a slot of red2 or xs is rewritten only after a later barrier has
+// ordered every read of it.
 __device__ __forceinline__ WalkPart cluster_sum2(cg::cluster_group& cl, float a, float b,
-                                                 WalkPart* xs, int slot, float* red,
+                                                 WalkPart* xs, int slot, WalkPart (*red2)[32],
                                                  WalkPart* bcast) {
-  a = block_sum<kWalkThreads>(a, red);
-  b = block_sum<kWalkThreads>(b, red);
-  if (threadIdx.x == 0) xs[slot] = WalkPart{a, b};
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  a = warp_sum(a);
+  b = warp_sum(b);
+  if (lane == 0) red2[slot][warp] = WalkPart{a, b};
+  __syncthreads();
+  if (warp == 0) {
+    WalkPart v = lane < kWalkThreads / 32 ? red2[slot][lane] : WalkPart{0.f, 0.f};
+    v.a = warp_sum(v.a);
+    v.b = warp_sum(v.b);
+    if (lane == 0) xs[slot] = v;
+  }
   cl.sync();
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
+  if (warp == 0) {
     WalkPart v{0.f, 0.f};
     if (lane < (int)cl.num_blocks()) v = *cl.map_shared_rank(&xs[slot], lane);
 #pragma unroll
@@ -335,12 +326,16 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ float red[32];
   __shared__ int32_t redi[32];
-  __shared__ int kids[64];
   __shared__ int32_t s_removed[64];  // tokens of the rejected siblings, in order
-  __shared__ int s_nk, s_acc;
-  __shared__ float s_lse;
   __shared__ int32_t s_tok[64], s_par[64], s_rank[64];
+  // per target row r (0 = root, r = node r - 1): log-sum-exp of t_r / T, the
+  // node's children in rank order, and the first child if its coin accepts
+  __shared__ float s_lse_row[65];
+  __shared__ int8_t s_kid[65][64];
+  __shared__ int s_nkid[65];
+  __shared__ int s_first_acc[65];
   __shared__ WalkPart xs[2], bcast;
+  __shared__ WalkPart red2[2][32];
   __shared__ float x_best;
   __shared__ int32_t x_bid;
   int n = w.n_nodes[b];
@@ -348,13 +343,63 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
     if (tid == 0 && rank == 0) set_status(w.status, DT_EDEVICE);
     n = n < 0 ? 0 : w.Nmax;
   }
+  const int V = w.V;
   for (int i = tid; i < n; i += kWalkThreads) {
-    s_tok[i] = w.tokens[(size_t)b * w.Nmax + i];
+    int tok = w.tokens[(size_t)b * w.Nmax + i];
+    if (tok < 0 || tok >= V) {  // range check: the walk indexes rows by token
+      if (rank == 0) set_status(w.status, DT_EDEVICE);
+      tok = 0;
+    }
+    s_tok[i] = tok;
     s_par[i] = w.parents[(size_t)b * w.Nmax + i];
     s_rank[i] = w.ranks[(size_t)b * w.Nmax + i];
   }
+  for (int r0 = tid; r0 <= n; r0 += kWalkThreads) s_nkid[r0] = 0;
   __syncthreads();
-  const int V = w.V;
+  // Everything the walk needs per node that does not depend on the path
+  // taken, for all rows at once: the rows' log-sum-exp (one warp per row,
+  // from the pre-pass's split partials), the children in rank order (ties
+  // to the lower index, as a stable sort gives), and the coin of each
+  // node's first child, which meets p and q before any residual.
+  for (int r0 = warp; r0 <= n; r0 += kWalkThreads / 32) {
+    const size_t rg = (size_t)b * (w.Nmax + 1) + r0;
+    float m2 = -INFINITY;
+    for (int s = lane; s < w.splits; s += 32) m2 = fmaxf(m2, w.parts.pv[rg * w.splits + s]);
+    m2 = warp_max(m2);
+    float s2 = 0.f;
+    for (int s = lane; s < w.splits; s += 32) {
+      const float mv = w.parts.pv[rg * w.splits + s];
+      if (mv != -INFINITY) s2 += w.parts.ps[rg * w.splits + s] * exp2f((mv - m2) * kL2e);
+    }
+    s2 = warp_sum(s2);
+    if (lane == 0) s_lse_row[r0] = m2 + logf(s2);
+  }
+  for (int c = tid; c < n; c += kWalkThreads) {
+    const int p = s_par[c];
+    if (p < -1 || p >= n) continue;  // a child of no node the walk can visit
+    int pos = 0;
+    for (int j = 0; j < n; ++j)
+      pos += (s_par[j] == p && (s_rank[j] < s_rank[c] || (s_rank[j] == s_rank[c] && j < c))) ? 1
+                                                                                            : 0;
+    s_kid[p + 1][pos] = (int8_t)c;
+    atomicAdd(&s_nkid[p + 1], 1);
+  }
+  __syncthreads();
+  const float temp = w.temp;
+  for (int r0 = tid; r0 <= n; r0 += kWalkThreads) {
+    int acc = -1;
+    if (s_nkid[r0] > 0) {
+      const int c = s_kid[r0][0];
+      const int x = s_tok[c];
+      const size_t rg = (size_t)b * (w.Nmax + 1) + r0;
+      const float px = expf(__fdiv_rn(ld_logit(w.t, w.tbf16, rg * V + x), temp) - s_lse_row[r0]);
+      const float qx = w.draft_q[rg * V + x] / 1.f;
+      const float u = philox_uniform(w.seed, w.offset, 1u, (uint32_t)b, (uint32_t)c, 0u, 0u);
+      if (u < px / qx) acc = c;
+    }
+    s_first_acc[r0] = acc;
+  }
+  __syncthreads();
   // Vector mode: rows of a multiple of 4 tokens on 16-byte boundaries, read
   // and written four tokens per load; every slice starts on a multiple of 4.
   const bool vec = (V & 3) == 0 && ((uintptr_t)w.t & 15) == 0 && ((uintptr_t)w.draft_q & 15) == 0 &&
@@ -362,90 +407,72 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
   const int sh = vec ? 2 : 0;  // log2 of the tokens a thread reads at once
   const int chunk = vec ? ((V + 4 * C - 1) / (4 * C)) * 4 : (V + C - 1) / C;
   const int v0 = min(V, rank * chunk), v1 = min(V, v0 + chunk);  // this CTA's slice
-  const float temp = w.temp;
   float* rb[2] = {w.rbuf + (size_t)b * 2 * V, w.rbuf + (size_t)b * 2 * V + V};
   int node = -1, nacc = 0, slot = 0;
   int32_t bonus = 0;
+  // Residual buffer holding p (unnormalised) while `resid`.  It carries over
+  // from node to node: a node's first pass writes the other buffer, so it
+  // never overwrites what a slower CTA may still read for the previous
+  // node's last coin (the pass after it follows a cluster barrier).
+  int cur = 0;
   while (true) {
     const int row = node + 1;
     const size_t rg = (size_t)b * (w.Nmax + 1) + row;
-    if (warp == 0) {
-      float m2 = -INFINITY;
-      for (int s = lane; s < w.splits; s += 32) m2 = fmaxf(m2, w.parts.pv[rg * w.splits + s]);
-      m2 = warp_max(m2);
-      float s2 = 0.f;
-      for (int s = lane; s < w.splits; s += 32) {
-        const float mv = w.parts.pv[rg * w.splits + s];
-        if (mv != -INFINITY) s2 += w.parts.ps[rg * w.splits + s] * exp2f((mv - m2) * kL2e);
-      }
-      s2 = warp_sum(s2);
-      if (lane == 0) {
-        s_lse = m2 + logf(s2);
-        int c = 0;
-        for (int i = 0; i < n; ++i)
-          if (s_par[i] == node) kids[c++] = i;
-        for (int i = 1; i < c; ++i) {  // insertion sort by rank (at most k entries)
-          const int v = kids[i];
-          int j = i - 1;
-          while (j >= 0 && s_rank[kids[j]] > s_rank[v]) {
-            kids[j + 1] = kids[j];
-            --j;
-          }
-          kids[j + 1] = v;
-        }
-        s_nk = c;
-        s_acc = -1;
-      }
-    }
-    __syncthreads();
-    const float lse_t = s_lse;
-    const int nk = s_nk;
+    const float lse_t = s_lse_row[row];
+    const int nk = s_nkid[row];
     const size_t tbase = rg * V;
     const float* q = w.draft_q + rg * V;
     bool resid = false;  // p is softmax(t / T) until the first effective residual
-    int cur = 0;         // residual buffer holding p (unnormalised) when resid
     float zr = 1.f;      // normaliser of the residual
     float qn = 1.f;      // sum of q over the tokens not yet removed
-    // The removed set is the first n_removed entries of s_removed (at most nk,
-    // and a node has fewer than Nmax <= 64 children).  A pass looks up the
-    // removed tokens that fall in this thread's groups of the slice (group g
-    // = (y - v0) >> sh belongs to thread g % kWalkThreads) only when it
-    // reaches the previous one, and meets them in ascending order as y
+    // The removed set is the sibling being rejected (xr) and the first
+    // n_removed entries of s_removed, the siblings rejected before it (fewer
+    // than nk, and a node has fewer than Nmax <= 64 children).  A pass looks
+    // up the removed tokens that fall in this thread's groups of the slice
+    // (group g = (y - v0) >> sh belongs to thread g % kWalkThreads) only when
+    // it reaches the previous one, and meets them in ascending order as y
     // advances.
     int n_removed = 0;
-    auto next_owned = [&](int after) {
-      int best = 0x7fffffff;
+    auto next_owned = [&](int after, int xr) {
+      auto mine = [&](int t) {
+        return t > after && t >= v0 && t < v1 && ((t - v0) >> sh) % kWalkThreads == tid;
+      };
+      int best = mine(xr) ? xr : 0x7fffffff;
       for (int i = 0; i < n_removed; ++i) {
         const int t = s_removed[i];
-        if (t > after && t >= v0 && t < v1 && ((t - v0) >> sh) % kWalkThreads == tid)
-          best = min(best, t);
+        if (mine(t)) best = min(best, t);
       }
       return best;
     };
+    int acc = -1;
     for (int ci = 0; ci < nk; ++ci) {
-      const int c = kids[ci];
+      const int c = s_kid[row][ci];
       const int x = s_tok[c];
-      const float px = resid ? __ldcg(rb[cur] + x) / zr : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + x), temp) - lse_t);
-      const float qx = q[x] / qn;
-      const float u = philox_uniform(w.seed, w.offset, 1u, (uint32_t)b, (uint32_t)c, 0u, 0u);
-      if (u < px / qx) {
-        if (tid == 0) s_acc = c;
+      bool take;
+      if (ci == 0) {
+        take = s_first_acc[row] >= 0;
+      } else {
+        const float px = resid ? __ldcg(rb[cur] + x) / zr
+                               : expf(__fdiv_rn(ld_logit(w.t, w.tbf16, tbase + x), temp) - lse_t);
+        const float qx = q[x] / qn;
+        const float u = philox_uniform(w.seed, w.offset, 1u, (uint32_t)b, (uint32_t)c, 0u, 0u);
+        take = u < px / qx;
+      }
+      if (take) {
+        acc = c;
         break;  // uniform over the cluster: every thread computed the same values
       }
       // residual pass over this CTA's slice: r'(y) = max(p(y) - q_j(y), 0),
       // q_j = q without the tokens removed before x, over the normaliser qn
-      if (tid == 0) s_removed[n_removed] = x;
-      ++n_removed;
-      __syncthreads();
       float* dst = rb[cur ^ 1];
       float zsum = 0.f, qsum = 0.f;
-      int nxt = next_owned(-1);
+      int nxt = next_owned(-1, x);
       // one token: p(y), then r'(y) = max(p(y) - q_j(y), 0) with q_j(y) = 0
       // for tokens removed before x, over the normaliser qn
       auto resid_one = [&](int y, float praw, float qv) {
         const float py = resid ? praw / zr : expf(__fdiv_rn(praw, temp) - lse_t);
         const bool rm = (y == nxt);
-        if (rm) nxt = next_owned(y);
+        if (rm) nxt = next_owned(y, x);
         const float rv = fmaxf(py - (rm && y != x ? 0.f : qv) / qn, 0.f);
         zsum += rv;
         if (!rm) qsum += qv;
@@ -487,7 +514,11 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
         for (int y = v0 + tid; y < v1; y += kWalkThreads)
           dst[y] = resid_one(y, resid ? rb[cur][y] : ld_logit(w.t, w.tbf16, tbase + y), q[y]);
       }
-      const WalkPart tot = cluster_sum2(cl, zsum, qsum, xs, slot, red, &bcast);
+      // x joins the removed set for the next pass: no thread reads this entry
+      // before the barriers of the reduction below
+      if (tid == 0) s_removed[n_removed] = x;
+      ++n_removed;
+      const WalkPart tot = cluster_sum2(cl, zsum, qsum, xs, slot, red2, &bcast);
       slot ^= 1;
       if (tot.a > 0.f) {
         cur ^= 1;
@@ -496,13 +527,10 @@ __global__ void __launch_bounds__(kWalkThreads) stoch_walk_kernel(WalkArgs w) {
       }
       qn = tot.b;
     }
-    __syncthreads();
-    const int acc = s_acc;
     if (acc >= 0 && nacc < w.Bk) {
       if (tid == 0 && rank == 0) w.acc_nodes[(size_t)b * w.Bk + nacc] = acc;
       ++nacc;
       node = acc;
-      __syncthreads();
       continue;
     }
     // bonus: exponential race argmax_y p(y) / E_y over every slice

@@ -52,7 +52,8 @@ namespace dt {
 // cost): quadrant q holds node group q % (NT / 32) of replica q / (NT / 32).
 // Epilogue warps 0-7 (two per quadrant) split a tile's 256 columns: the
 // 2R warps that see the same node group take one part of 256 / (2R) = NT
-// columns each.
+// columns each.  NT is the kernel's capacity (32 or 64 rows); a wave of the
+// 64-row kernel with at most 32 rows uses the 32-row layout (four replicas).
 template <int NG>
 struct PShape {
   static constexpr int NT = 32 * NG;          // node rows per replica
@@ -86,7 +87,8 @@ struct PMeta {
 // device (offsets).  Offsets are from a 1024-byte aligned base.
 //
 // The A operand: chunk kc (K columns 64 kc .. 64 kc + 63) of A row i at
-// a + (kc * 128 + i) * 128, 128-byte swizzled; A row i holds node i % NT.
+// a + (kc * 128 + i) * 128, 128-byte swizzled; A row i holds node i % nte,
+// nte = 32 or 64 the node rows per replica of the wave.
 struct PLayout {
   size_t a, bias, lists, cands, sorted, keys, rlse, rlq, rtok, spos, spar, msv, msi, misc, req,
       rows0, rows1, meta, exch, bars, flags, stage, total;
@@ -710,6 +712,15 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
       const int n_rows = misc[5];
       if (n_rows == 0 || misc[6]) break;  // uniform (shared memory after a barrier)
       Row* rows = rows_buf[cur];
+      // A wave of at most 32 node rows runs in the one-group layout even in
+      // the 64-row kernel: its rows replicated four times, so that all eight
+      // epilogue warps share 32 nodes instead of half of them idling on an
+      // empty second node group.
+      const int ge = (NG == 2 && n_rows > 32) ? 2 : 1;  // node groups of this wave
+      const int nte = 32 * ge;                          // node rows per replica
+      const int re = 4 / ge;                            // replicas down the 128 A rows
+      const int parts = 2 * re;                         // column parts per node group
+      const int pcols = S::kTileN / parts;              // columns per part (= nte)
       // ---- this wave's node rows, and their Markov rows A[token] as the A operand
       for (int c = ct; c < NT; c += NCT) {
         PMeta m;
@@ -735,10 +746,10 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
       }
       named_bar(1, NCT);
       {
-        // rows 0 .. NT-1 of every chunk from global memory
-        const int npieces = KC * NT * 8;
+        // rows 0 .. nte-1 of every chunk from global memory
+        const int npieces = KC * nte * 8;
         for (int idx = ct; idx < npieces; idx += NCT) {
-          const int ch = idx & 7, c = (idx >> 3) % NT, kc = (idx >> 3) / NT;
+          const int ch = idx & 7, c = (idx >> 3) % nte, kc = (idx >> 3) / nte;
           const int col_k = kc * 64 + ch * 8;
           const int tok = c < n_rows ? rows[c].token : -1;
           const bool ok = meta[c].valid && tok >= 0 && col_k < a.r;
@@ -753,16 +764,16 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
       }
       named_bar(1, NCT);
       {
-        // A row i (of 128) is node i % NT: the replicas are byte copies of
-        // rows 0 .. NT-1 (NT is a multiple of the 8-row swizzle period)
-        constexpr int per = NT * 128 / 16;  // 16-byte pieces of one replica of a chunk
-        const int n = KC * (S::R - 1) * per;
+        // A row i (of 128) is node i % nte: the replicas are byte copies of
+        // rows 0 .. nte-1 (nte is a multiple of the 8-row swizzle period)
+        const int per = nte * 128 / 16;  // 16-byte pieces of one replica of a chunk
+        const int n = KC * (re - 1) * per;
         for (int idx = ct; idx < n; idx += NCT) {
-          const int kc = idx / ((S::R - 1) * per);
-          const int rr = 1 + (idx / per) % (S::R - 1);
+          const int kc = idx / ((re - 1) * per);
+          const int rr = 1 + (idx / per) % (re - 1);
           const int pc = idx % per;
           const uint4* src = (const uint4*)(aop + (size_t)kc * 128 * 128) + pc;
-          uint4* dst = (uint4*)(aop + (size_t)kc * 128 * 128 + (size_t)rr * NT * 128) + pc;
+          uint4* dst = (uint4*)(aop + (size_t)kc * 128 * 128 + (size_t)rr * nte * 128) + pc;
           *dst = *src;
         }
         // the tensor cores read these bytes through the async proxy
@@ -815,8 +826,8 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
         // cache, 1/T, an online max / sum-exp, the top-k of s (ties to the
         // lower token) and, at T > 0, the Gumbel-top-k of s + G.
         const int q = warp & 3;
-        const int c = 32 * (q % NG) + lane;
-        const int part = (q / NG) * 2 + (warp >> 2);
+        const int c = 32 * (q % ge) + lane;
+        const int part = (q / ge) * 2 + (warp >> 2);
         const float temp = a.temp;
         const PMeta mc = meta[c];
         const bool any = __any_sync(0xffffffffu, mc.valid) != 0;
@@ -838,12 +849,12 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           // the 128-row tile at the end of an odd range has columns 0-127 only
-          const bool has_part = !(odd && j == n_mt - 1) || part * S::kPartCols < kTileV;
+          const bool has_part = !(odd && j == n_mt - 1) || part * pcols < kTileV;
           if (any && has_part) {
 #pragma unroll 1
-            for (int c4 = 0; c4 < S::kPartCols / 32; ++c4) {
+            for (int c4 = 0; c4 < pcols / 32; ++c4) {
               __syncwarp();
-              const int col = part * S::kPartCols + 32 * c4;  // within the tile
+              const int col = part * pcols + 32 * c4;  // within the tile
               const int xq = (t0 + 2 * j) * kTileV + col;    // first token of the block
               const int nv = min(32, a.V - xq);
               float acc[32];
@@ -958,7 +969,7 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
         // thread per node merges them into the CTA's partial of the node
         constexpr int kEx = 2 + 2 * KMAX * (STOCH ? 2 : 1);  // words per (part, node)
         {
-          float* mine = exch + ((size_t)part * NT + c) * kEx;
+          float* mine = exch + ((size_t)part * nte + c) * kEx;
           mine[0] = m;
           mine[1] = ssum;
 #pragma unroll
@@ -973,15 +984,15 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
         }
         named_bar(2, S::kEpiWarps * 32);
         const int cn = threadIdx.x;  // node merged by this thread
-        if (cn < NT && meta[cn].valid) {
+        if (cn < nte && meta[cn].valid) {
           const int par = wave & 1;
           float mx = -INFINITY;
-          for (int pp = 0; pp < S::kParts; ++pp)
-            mx = fmaxf(mx, exch[((size_t)pp * NT + cn) * kEx]);
+          for (int pp = 0; pp < parts; ++pp)
+            mx = fmaxf(mx, exch[((size_t)pp * nte + cn) * kEx]);
           float sv = 0.f;
           if (mx != -INFINITY)
-            for (int pp = 0; pp < S::kParts; ++pp) {
-              const float* e = exch + ((size_t)pp * NT + cn) * kEx;
+            for (int pp = 0; pp < parts; ++pp) {
+              const float* e = exch + ((size_t)pp * nte + cn) * kEx;
               if (e[0] != -INFINITY) sv += e[1] * exp2f((e[0] - mx) * kLog2e);
             }
           a.pstats[par][(size_t)cn * ncta + cx] = make_float2(mx, sv);
@@ -989,18 +1000,19 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
             float* OV = (lst ? a.pgv[par] : a.plv[par]) + (size_t)cn * k * ncta + cx;
             int32_t* OI = (lst ? a.pgi[par] : a.pli[par]) + (size_t)cn * k * ncta + cx;
             const int off = 2 + (lst ? 2 * KMAX : 0);
-            int hd[S::kParts];  // heads of the parts' sorted lists
+            constexpr int kPartsMax = 8;  // parts of the one-group layout
+            int hd[kPartsMax];            // heads of the parts' sorted lists
 #pragma unroll
-            for (int pp = 0; pp < S::kParts; ++pp) hd[pp] = 0;
+            for (int pp = 0; pp < kPartsMax; ++pp) hd[pp] = 0;
             for (int i = 0; i < k; ++i) {
               int bw = 0;
               float bv = -INFINITY;
               int32_t bi = 0x7fffffff;
               bool have = false;
 #pragma unroll
-              for (int pp = 0; pp < S::kParts; ++pp) {
-                if (hd[pp] >= k) continue;
-                const float* e = exch + ((size_t)pp * NT + cn) * kEx + off;
+              for (int pp = 0; pp < kPartsMax; ++pp) {
+                if (pp >= parts || hd[pp] >= k) continue;
+                const float* e = exch + ((size_t)pp * nte + cn) * kEx + off;
                 const float v = e[hd[pp]];
                 const int32_t id = __float_as_int(e[KMAX + hd[pp]]);
                 if (!have || ranks_first(v, id, bv, bi)) {
@@ -1011,7 +1023,7 @@ __global__ void __launch_bounds__(PShape<NG>::kThreads, 1)
                 }
               }
 #pragma unroll
-              for (int pp = 0; pp < S::kParts; ++pp) hd[pp] += (pp == bw) ? 1 : 0;
+              for (int pp = 0; pp < kPartsMax; ++pp) hd[pp] += (pp == bw) ? 1 : 0;
               OV[(size_t)i * ncta] = bv;
               OI[(size_t)i * ncta] = bi;
             }

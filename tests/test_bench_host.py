@@ -88,3 +88,18 @@ def test_traffic_is_read_only_for_the_profiled_source(tmp_path, monkeypatch):
     assert bench.traffic_from_profile(str(src), name) is None
     # each kernel source has its own summary
     assert bench.PROFILE_OF["pbuild.cu"] == "pbuild_qwen3_4b.txt"
+
+
+def test_build_roofline_counts_bm_once_and_reports_the_stream():
+    """The roofline charges the Markov factor once per build; the stream
+    object counts one pass over it per wave."""
+    sys.path.insert(0, ROOT)
+    import bench
+    kern = {"pbuild": {"avg_us": 100.0}}
+    V, r = 1000, 64
+    roof = bench.build_roofline(kern, V=V, r=r, B=2, Bk=5, inner=9, lbytes=2, waves=4)
+    assert roof["algorithmic_bytes_per_launch"] == V * r * 2 + 2 * 5 * V * 2 + 9 * r * 2
+    assert roof["stream"]["bytes_per_launch"] == 4 * V * r * 2
+    assert abs(roof["stream"]["achieved_gbs"] - 4 * V * r * 2 / 100e-6 / 1e9) < 0.1
+    assert "stream" not in bench.build_roofline({"markov_gemm": {"avg_us": 10.0}}, V=V, r=r,
+                                                B=2, Bk=5, inner=9, lbytes=2, waves=4)
