@@ -66,6 +66,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--copies", type=int, default=4)
     p.add_argument("--no-oracle", action="store_true", help="skip the cpu_baseline leg")
+    p.add_argument("--attn-layers", type=int, default=36,
+                   help="also time the round with the verify attention run for this many target "
+                        "layers (Qwen3-4B and -8B have 36); 1 skips that leg")
     p.add_argument("--workload", default=WORKLOAD, choices=["qwen3_4b", "qwen3_8b", "load_adaptive", "treeflash", "acceptance_study", "load_policy", "calibration"])
     return p.parse_args()
 
@@ -551,6 +554,56 @@ def run_ours(args):
            "path": "python API (eager launches) + pinned H2D/D2H copies; the target rows "
                    "are copied on a second stream beside build and verify"}
 
+    # ---- the round with the verify attention run once per target layer.
+    # Every layer has its own Q and K/V buffers (the same values), so no layer
+    # finds another layer's K/V in L2.
+    attn_layers = None
+    if args.attn_layers > 1:
+        nl = args.attn_layers
+        lay = [{nm: copies[0][nm].clone() for nm in ("q", "kp", "vp", "kt", "vt")}
+               for _ in range(nl)]
+
+        def round_layers(c):
+            build(c)
+            for lb in lay:
+                dt.tree_verify_attn(lb["q"], lb["kp"], lb["vp"], c["pstart"], c["plen"], P,
+                                    lb["kt"], lb["vt"], tree.anc, tree.n_nodes, scale, attn_out,
+                                    ws_v)
+            accept_(c)
+
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                round_layers(copies[i % len(copies)])
+        torch.cuda.synchronize()
+        graphs_l = []
+        for c in copies:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                round_layers(c)
+            graphs_l.append(g)
+        kl = min(args.steps, 50)
+        with torch.cuda.stream(stream):
+            for i in range(max(args.warmup, 3)):
+                graphs_l[i % len(graphs_l)].replay()
+        torch.cuda.synchronize()
+        barrier()
+        e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e4.record(stream)
+            for i in range(kl):
+                graphs_l[i % len(graphs_l)].replay()
+            e5.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_l = max_over_ranks(e4.elapsed_time(e5), world, dev)
+        for wsx in (ws_b, ws_v, ws_a):
+            assert dt.read_status(wsx) == 0
+        attn_layers = {"layers": nl, "value": round(job_throughput(kl, world, ms_l), 1),
+                       "unit": UNIT, "ms_per_step": round(ms_l / kl, 5), "steps": kl,
+                       "how": "build + verify attention once per layer (own Q/K/V buffers per "
+                              "layer) + accept, CUDA graph per input copy"}
+        del graphs_l, lay
+
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5),
@@ -568,6 +621,8 @@ def run_ours(args):
         "clocks": clk,
         "tree_nodes": n,
     }
+    if attn_layers:
+        out["attention_x_layers"] = attn_layers
     if rank == 0 and world == 1 and not args.no_oracle and args.workload == WORKLOAD:
         v, nr, el = time_oracle(w, tgt[0], budget_s=20.0)
         vc, nc, elc = time_cpu_round(w, tgt[0], budget_s=10.0)
