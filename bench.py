@@ -318,6 +318,41 @@ def build_roofline(kern, *, V, r, B, Bk, inner, lbytes, waves=None):
     return roof
 
 
+def round_roofline(value, world, *, build_bytes, build_flops, prefix_lens, n_nodes, inner, V,
+                   Hq, Hkv, d, tbytes, temp):
+    """Roofline of the whole round: the sum over its three calls of
+    max(algorithmic bytes / HBM bandwidth, algorithmic flops / dense bf16).
+
+    Per request b with n_b nodes and prefix P_b:
+      build   the build's bytes and flops (the Markov factor once, see
+              build_roofline), plus at T > 0 the fp32 draft-q rows it writes
+              (`inner` rows of V);
+      verify  K and V of P_b + n_b + 1 columns (bf16), Q read and O written
+              for n_b + 1 rows; 4 (n_b + 1) Hq d (P_b + n_b + 1) flops;
+      accept  the n_b + 1 target rows, read once (the T > 0 residual passes
+              depend on the draws and are not counted).
+    `value` is the job's rounds/s over `world` GPUs; frac compares one GPU's
+    share with the one-GPU bound.
+    """
+    pk, pk_kind = peaks()
+    bw = pk["hbm_gbs"] * 1e9
+    tf = pk["bf16_tflops"] * 1e12
+    rows = np.asarray(n_nodes, np.float64) + 1.0
+    cols = np.asarray(prefix_lens, np.float64) + rows
+    qbytes = inner * V * 4.0 if temp > 0 else 0.0
+    vbytes = float((cols * Hkv * d * 2 * 2).sum() + (rows * Hq * d * 2 * 2).sum())
+    vflops = float((4.0 * rows * Hq * d * cols).sum())
+    abytes = float((rows * V * tbytes).sum())
+    t = {"build": max((build_bytes + qbytes) / bw, build_flops / tf),
+         "verify": max(vbytes / bw, vflops / tf),
+         "accept": abytes / bw}
+    t_round = sum(t.values())
+    return {"bytes_per_round": int(build_bytes + qbytes + vbytes + abytes),
+            "us_at_roofline": {k: round(v * 1e6, 2) for k, v in t.items()},
+            "rounds_per_s_at_roofline": round(1.0 / t_round, 1),
+            "frac": round(value / world * t_round, 4), "peak_kind": pk_kind}
+
+
 # ncu summary of each kernel source's launch on the headline workload
 PROFILE_OF = {"markov_gemm.cu": "markov_gemm_qwen3_4b.txt", "pbuild.cu": "pbuild_qwen3_4b.txt"}
 
@@ -623,6 +658,11 @@ def run_ours(args):
     }
     if attn_layers:
         out["attention_x_layers"] = attn_layers
+    out["round_roofline"] = round_roofline(
+        value, world,
+        build_bytes=V * r * 2 + B * Bk * V * (2 if w.logit_dtype == "bf16" else 4) + inner * r * 2,
+        build_flops=2.0 * inner * V * r, prefix_lens=w.prefix_len, n_nodes=n_nodes, inner=inner,
+        V=V, Hq=w.Hq, Hkv=w.Hkv, d=w.d, tbytes=2 if w.logit_dtype == "bf16" else 4, temp=temp)
     if rank == 0 and world == 1 and not args.no_oracle and args.workload == WORKLOAD:
         v, nr, el = time_oracle(w, tgt[0], budget_s=20.0)
         vc, nc, elc = time_cpu_round(w, tgt[0], budget_s=10.0)

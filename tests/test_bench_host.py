@@ -103,3 +103,29 @@ def test_build_roofline_counts_bm_once_and_reports_the_stream():
     assert abs(roof["stream"]["achieved_gbs"] - 4 * V * r * 2 / 100e-6 / 1e9) < 0.1
     assert "stream" not in bench.build_roofline({"markov_gemm": {"avg_us": 10.0}}, V=V, r=r,
                                                 B=2, Bk=5, inner=9, lbytes=2, waves=4)
+
+
+def test_round_roofline_sums_the_three_calls():
+    """Round roofline: build + verify + accept bytes (and flops where they
+    bind) at the peak; the headline shape gives ~99 MB per round."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    V, r = 151936, 256
+    build_bytes = V * r * 2 + 7 * V * 2 + 27 * r * 2
+    rr = bench.round_roofline(1000.0, 1, build_bytes=build_bytes, build_flops=2.0 * 27 * V * r,
+                              prefix_lens=np.array([2048]), n_nodes=np.array([32]), inner=27,
+                              V=V, Hq=32, Hkv=8, d=128, tbytes=2, temp=0.0)
+    kv = (2048 + 33) * 8 * 128 * 2 * 2
+    qo = 33 * 32 * 128 * 2 * 2
+    assert rr["bytes_per_round"] == build_bytes + kv + qo + 33 * V * 2
+    pk, _ = bench.peaks()
+    t = rr["bytes_per_round"] / (pk["hbm_gbs"] * 1e9)
+    assert abs(rr["rounds_per_s_at_roofline"] - 1.0 / t) / (1.0 / t) < 1e-3
+    assert abs(rr["frac"] - 1000.0 * t) < 1e-3
+    # at T > 0 the build also writes its fp32 q rows; two GPUs double the job rate
+    r2 = bench.round_roofline(2000.0, 2, build_bytes=build_bytes, build_flops=0.0,
+                              prefix_lens=np.array([2048]), n_nodes=np.array([32]), inner=27,
+                              V=V, Hq=32, Hkv=8, d=128, tbytes=2, temp=0.6)
+    assert r2["bytes_per_round"] == rr["bytes_per_round"] + 27 * V * 4
+    assert r2["frac"] > rr["frac"]
