@@ -244,7 +244,12 @@ dt_status dt_tree_verify_attn(const void* d_q, const void* d_k_prefix,
  *   removed, renormalised.  With no child accepted, or at a leaf, the bonus is
  *   argmax_x p(x) / E_x, E_x = -log U'_x (Philox purpose 2).
  *   d_target_logits [batch][Nmax+1][V] fp32 or bf16, row 0 = root, row i+1 =
- *   node i; tree = the dt_tree of dt_tree_build (d_draft_q needed iff T > 0).
+ *   node i; tree = the dt_tree of dt_tree_build, or any tree in its layout
+ *   (d_draft_q needed iff T > 0).  A node may have any number of children
+ *   (up to Nmax - 1), taken in rank order with equal ranks in node order.
+ *   At T > 0 a token outside [0, V) records DT_EDEVICE in the status word and
+ *   reads as token 0; a node whose parent is outside [-1, n) is never
+ *   reached.
  * Outputs (device): d_acc_nodes [batch][Bk] accepted node indices by depth
  * (-1 padded), d_n_acc [batch], d_bonus [batch].
  * At T > 0 each request's walk runs on one thread-block cluster of up to 8
