@@ -353,8 +353,9 @@ def round_roofline(value, world, *, build_bytes, build_flops, prefix_lens, n_nod
             "frac": round(value / world * t_round, 4), "peak_kind": pk_kind}
 
 
-# ncu summary of each kernel source's launch on the headline workload
-PROFILE_OF = {"markov_gemm.cu": "markov_gemm_qwen3_4b.txt", "pbuild.cu": "pbuild_qwen3_4b.txt"}
+# ncu summary of each kernel source's launch on the workload where it dominates
+# (the per-wave GEMM: the 64-request batch); a missing summary reads as unknown
+PROFILE_OF = {"markov_gemm.cu": "markov_gemm_load_adaptive.txt", "pbuild.cu": "pbuild_qwen3_4b.txt"}
 
 
 def traffic_from_profile(kernel_src, profile=None):
